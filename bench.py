@@ -1,0 +1,337 @@
+#!/usr/bin/env python3
+"""Benchmark: batch-1 greedy decode tokens/s of the ~1.9B (2B-class) bf16 decoder at a
+4096-token context on one B200, and the fraction of the HBM roofline it reaches.
+
+A step is one whole decode run of the workload (kd_reset + one kd_decode launch that
+generates n_gen tokens, i.e. every row of the hot path, n_gen times). Weights, KV cache and
+the start token are resident in HBM before timing starts; timing uses CUDA events on the
+decode stream, max over ranks. The model streams 3.65 GB of weights per token, far above
+the 126 MB L2, so no flush is needed between steps.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+With --gpus N > 1 (launched under torch.distributed.run) each rank runs an independent
+replica of the request on its own GPU: batch-1 decode has no data-parallel split, so the
+aggregate is N replicas ("weak" scaling), with no collective on the data path.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "batch-1 decode tokens/s on 1 B200 (2B bf16) and % of HBM-bandwidth roofline"
+SPEC_HBM_GBS = 8000.0          # B200 HBM3e specification
+FALLBACK_HBM_GBS = 6650.0       # earlier measurement on this machine, if no measured peaks file
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="2b-4k")
+    ap.add_argument("--n-gen", type=int, default=None, help="override generated tokens per step")
+    ap.add_argument("--impl", default="kernel", choices=["kernel", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-sample-tokens", type=int, default=8)
+    return ap.parse_args()
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi SM clock and throttle reasons, sampled every 200 ms while timing."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.Q, "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.t.join(timeout=2)
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def cpu_cores():
+    return os.cpu_count() or 1
+
+
+def run_oracle_sample(w, weights_h, K, V, start, n_tokens):
+    """Time the oracle (single-threaded) generating n_tokens of workload w; tokens/s."""
+    import oracle
+    o = oracle.Oracle(w.dims(), weights_h, capacity=w.start_pos + w.n_pending + n_tokens, n_threads=1)
+    if K is not None:
+        o.set_kv(K, V)
+    t0 = time.perf_counter()
+    o.greedy(start, w.start_pos, n_tokens, keep_logits=False)
+    dt = time.perf_counter() - t0
+    o.close()
+    return n_tokens / dt, dt
+
+
+def lscpu_model():
+    try:
+        out = subprocess.run(["lscpu"], capture_output=True, text=True, timeout=10).stdout
+        for ln in out.splitlines():
+            if ln.startswith("Model name"):
+                return ln.split(":", 1)[1].strip()
+    except Exception:
+        pass
+    return "unknown"
+
+
+def reference_arm(args, w):
+    """The oracle, as it stands, timed on the host cores; rank 0 only."""
+    import torch
+    import synth
+    rank, world, local = dist_env()
+    if rank != 0:
+        return
+    n_tok = 1  # tokens per step: one decode step of the full workload is ~2 s on one core
+    weights = synth.make_weights(w)
+    wh = {k: v.cpu() for k, v in weights.items()}
+    del weights
+    K = V = None
+    if w.kv_len:
+        K, V = synth.make_kv(w)
+        K, V = K.cpu(), V.cpu()
+    start = synth.make_prompt(w).numpy()
+    for _ in range(args.warmup):
+        run_oracle_sample(w, wh, K, V, start, n_tok)
+    total = 0.0
+    for _ in range(args.steps):
+        _, dt = run_oracle_sample(w, wh, K, V, start, n_tok)
+        total += dt
+    value = args.steps * n_tok / total
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic", "config": workload_config(w, n_tok),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                         "sample": "%d decode token(s) per step of workload %s (start token at position %d), "
+                                   "single-threaded oracle; host %s, %d cores present"
+                                   % (n_tok, w.name, w.start_pos, lscpu_model(), cpu_cores())},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(w, n_gen):
+    return {"workload": w.name, "n_layers": w.n_layers, "d_model": w.d_model, "n_heads": w.n_heads,
+            "n_kv_heads": w.n_kv_heads, "head_dim": w.head_dim, "ffn_dim": w.ffn_dim, "vocab": w.vocab,
+            "kv_len": w.kv_len, "prompt_len": w.prompt_len, "n_gen": n_gen, "batch": 1,
+            "parallelism": "replicas", "l2": "inputs larger than L2 (weights streamed every token)"}
+
+
+def main():
+    args = parse()
+    import synth
+    w = synth.get(args.workload)
+    if args.n_gen:
+        w = w.replace(n_gen=args.n_gen)
+    if args.impl == "reference":
+        return reference_arm(args, w)
+
+    import torch
+    import torch.distributed as dist
+    rank, world, local = dist_env()
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+
+    from persistent_monokernel_sm_b200 import build
+    build.build()
+    import persistent_monokernel_sm_b200 as kd
+
+    weights = synth.make_weights(w, device="cuda")
+    K = V = None
+    if w.kv_len:
+        K, V = synth.make_kv(w, device="cuda")
+    start = synth.make_prompt(w)
+    dec = kd.Decoder(w.dims(), w.capacity, device=dev)
+    dec.load_weights(weights)
+    if K is not None:
+        dec.set_kv(K, V)
+    weights_h = None
+    if rank == 0 and not args.no_cpu_baseline:
+        weights_h = {k: v.cpu() for k, v in weights.items()}
+        Kh, Vh = (K.cpu(), V.cpu()) if K is not None else (None, None)
+    del weights
+    torch.cuda.empty_cache()
+    stream = dec.stream
+    d_start = start.to(dev)
+    tok_out = torch.empty(w.n_gen, dtype=torch.int32, device=dev)
+
+    def step():
+        dec.reset(d_start, w.start_pos)
+        dec.decode(w.n_gen, out=tok_out)
+
+    for _ in range(args.warmup):
+        step()
+    dec.sync()
+    launches0 = dec.info().launches
+
+    # ---- device-timed region
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    with ClockSampler(dev.index if dev.index is not None else 0) as clk:
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for i in range(args.steps):
+            dec.reset(d_start, w.start_pos)
+            ev[i][0].record(stream)
+            dec.decode(w.n_gen, out=tok_out)
+            ev[i][1].record(stream)
+        t1.record(stream)
+        torch.cuda.synchronize(dev)
+    dec.sync()
+    total_ms = t0.elapsed_time(t1)
+    kern_ms = [a.elapsed_time(b) for a, b in ev]
+    launches = dec.info().launches - launches0
+    t = torch.tensor([total_ms, max(kern_ms)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        dist.barrier()
+    total_ms, kern_max = float(t[0]), float(t[1])
+
+    # ---- end to end through the public host-memory call
+    h_in = start.pin_memory()
+    h_out = torch.empty(w.n_gen, dtype=torch.int32).pin_memory()
+    dec.generate(h_in, w.start_pos, w.n_gen, h_out)  # warm
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        dec.generate(h_in, w.start_pos, w.n_gen, h_out)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
+    e2e_ms = float(e2e_ms[0])
+
+    # ---- roofline of the monokernel: algorithmic bytes per launch / launch time
+    cfg = dec.cfg
+    bytes_launch = sum(kd.kd_step_bytes(cfg, w.start_pos + i + 1, True) for i in range(w.n_steps))
+    mean_kern_ms = statistics.mean(kern_ms)
+    achieved = bytes_launch / (mean_kern_ms * 1e-3) / 1e9
+    peak, peak_kind = measured_peaks()
+
+    line = None
+    if rank == 0:
+        tokens = args.steps * w.n_gen * world
+        value = tokens / (total_ms * 1e-3)
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "storage": "bf16 weights and KV cache",
+            "data": "synthetic", "config": workload_config(w, w.n_gen),
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": None,
+                         "peak_source": "%s copy bandwidth (MEASURED_PEAKS.json hbm_gbs)" % peak_kind
+                         if peak_kind == "measured" else "fallback 6.65 TB/s",
+                         "frac_of_8tbs_spec": achieved / SPEC_HBM_GBS,
+                         "bytes_per_launch": bytes_launch, "kernel": "kd::monokernel",
+                         "launch_ms": mean_kern_ms},
+            "tokens_per_s_per_launch": w.n_gen / (mean_kern_ms * 1e-3),
+            "roofline_tokens_per_s": w.n_gen / (bytes_launch / (peak * 1e9)),
+            "e2e": {"value": args.steps * w.n_gen * world / (e2e_ms * 1e-3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": 4 * w.n_pending, "d2h_bytes_per_step": 4 * w.n_gen},
+            "gpu_launches": launches, "launches_per_token": launches / (args.steps * w.n_gen),
+            "clocks": clk.summary(),
+        }
+    if rank == 0 and not args.no_cpu_baseline:
+        n = max(1, args.cpu_sample_tokens)
+        tps, dt = run_oracle_sample(w, weights_h, Kh, Vh, start.numpy(), n)
+        line["cpu_baseline"] = {
+            "value": tps, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": "first %d greedy tokens of workload %s, single-threaded oracle, %.1f s; host %s, %d cores"
+                      % (n, w.name, dt, lscpu_model(), cpu_cores())}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    dec.close()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,448 @@
+// kd_api.cu -- host side of libkd: configuration checks, the arena layout, weight repacking
+// into the streaming layout, and the C ABI declared in include/kd.h.
+#include <cuda_runtime.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include "kd.h"
+#include "kd_layout.h"
+
+using namespace kd;
+
+namespace {
+
+constexpr int kMaxGrid = 256;  // partial-record room for up to this many CTAs
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+bool valid_config(const kd_config* c) {
+    if (!c) return false;
+    if (c->n_layers < 1 || c->d_model <= 0 || c->n_heads <= 0 || c->n_kv_heads <= 0) return false;
+    if (c->head_dim != 64 && c->head_dim != 128) return false;
+    if (c->n_heads % c->n_kv_heads || c->n_heads / c->n_kv_heads > kMaxGroup) return false;
+    if (c->n_kv_heads > kMaxKvHeads) return false;
+    if (c->d_model % 64 || c->ffn_dim <= 0 || c->ffn_dim % 64) return false;
+    if (4LL * c->d_model > kStageBytes || 2LL * c->ffn_dim > kStageBytes) return false;
+    if (2LL * c->n_heads * c->head_dim > kStageBytes) return false;
+    if (c->vocab < 1 || c->max_seq < 1) return false;
+    if (!(c->rms_eps >= 0.f) || !(c->rope_theta > 0.f)) return false;
+    return true;
+}
+
+Dims make_dims(const kd_config* c) {
+    Dims d;
+    d.L = c->n_layers, d.d = c->d_model, d.Hq = c->n_heads, d.Hkv = c->n_kv_heads, d.hd = c->head_dim;
+    d.F = c->ffn_dim, d.V = c->vocab, d.S = c->max_seq, d.eps = c->rms_eps, d.theta = c->rope_theta;
+    d.qd = d.Hq * d.hd, d.kvd = d.Hkv * d.hd, d.r = d.Hq / d.Hkv;
+    d.qkv_rows = d.qd + 2 * d.kvd;
+    return d;
+}
+
+Layout make_layout(const Dims& d) {
+    Layout y;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        size_t at = off;
+        off = align256(off + bytes);
+        return at;
+    };
+    const size_t D = d.d;
+    y.embed = take((size_t)d.V * D * 2);
+    y.lm_head = take((size_t)d.V * D * 2);
+    y.final_norm = take(D * 2);
+    y.layer0 = off;
+    size_t lo = 0;
+    auto ltake = [&](size_t bytes) {
+        size_t at = lo;
+        lo = align256(lo + bytes);
+        return at;
+    };
+    y.l_attn_norm = ltake(D * 2);
+    y.l_ffn_norm = ltake(D * 2);
+    y.l_wqkv = ltake((size_t)d.qkv_rows * D * 2);
+    y.l_wo = ltake(D * d.qd * 2);
+    y.l_wgu = ltake((size_t)2 * d.F * D * 2);
+    y.l_wd = ltake(D * d.F * 2);
+    y.layer_stride = lo;
+    off = y.layer0 + (size_t)d.L * y.layer_stride;
+    y.weights_end = off;
+    const size_t kv = (size_t)d.L * d.Hkv * d.S * d.hd * 2;
+    y.kcache = take(kv);
+    y.vcache = take(kv);
+    y.kv_bytes = 2 * kv;
+    y.x = take(D * 4);
+    y.q = take((size_t)d.qd * 4);
+    y.o = take((size_t)d.qd * 4);
+    y.hdn = take((size_t)d.F * 4);
+    y.part = take((size_t)kMaxGrid * d.r * (d.hd + 2) * 4);
+    y.ctl = take((size_t)kCtlWords * 8);
+    y.tokens_in = take((size_t)d.S * 4);
+    y.tokens_out = take((size_t)d.S * 4);  // staging for kd_generate
+    y.total = off;
+    return y;
+}
+
+}  // namespace
+
+struct kd_ctx {
+    kd_config cfg;
+    Dims dm;
+    Layout lay;
+    uint8_t* arena;
+    cudaStream_t stream;
+    int device;
+    int nb, smem, ns, pieces, pos_per_stage, xs_floats;
+    bool has_weights, failed;
+    int pos, n_pending;
+    long long launches;
+    long long timeout_ns;
+    unsigned long long* trace;
+    int trace_every, trace_rows;
+    char err[512];
+};
+
+static int fail(kd_ctx* c, int code, const char* fmt, ...) {
+    if (c) {
+        va_list ap;
+        va_start(ap, fmt);
+        vsnprintf(c->err, sizeof c->err, fmt, ap);
+        va_end(ap);
+    }
+    return code;
+}
+
+#define KD_CUDA(ctx, call)                                                                       \
+    do {                                                                                         \
+        cudaError_t e_ = (call);                                                                 \
+        if (e_ != cudaSuccess)                                                                   \
+            return fail((ctx), KD_ECUDA, "%s failed: %s", #call, cudaGetErrorString(e_));        \
+    } while (0)
+
+// ------------------------------------------------------------------ repack kernels
+
+namespace {
+
+// dst row r of the fused [q; k; v] projection: q and k heads hold RoPE pairs (i, i + hd/2)
+// in adjacent rows (2i, 2i + 1); v rows keep their order.
+__global__ void repack_qkv(uint8_t* dst_layer0, size_t layer_stride, size_t off, const uint16_t* wq,
+                           const uint16_t* wk, const uint16_t* wv, Dims dm) {
+    const int r = blockIdx.x, l = blockIdx.y;
+    const uint16_t* src;
+    int row;
+    if (r < dm.qd + dm.kvd) {
+        const bool isq = r < dm.qd;
+        const int rr = isq ? r : r - dm.qd;
+        const int h = rr / dm.hd, j = rr % dm.hd;
+        row = h * dm.hd + (j >> 1) + ((j & 1) ? dm.hd / 2 : 0);
+        src = isq ? wq + (size_t)l * dm.qd * dm.d : wk + (size_t)l * dm.kvd * dm.d;
+    } else {
+        row = r - dm.qd - dm.kvd;
+        src = wv + (size_t)l * dm.kvd * dm.d;
+    }
+    const uint4* s = reinterpret_cast<const uint4*>(src + (size_t)row * dm.d);
+    uint4* d = reinterpret_cast<uint4*>(dst_layer0 + (size_t)l * layer_stride + off + (size_t)r * dm.d * 2);
+    for (int i = threadIdx.x; i < dm.d / 8; i += blockDim.x) d[i] = s[i];
+}
+
+// dst rows (2i, 2i + 1) = (gate row i, up row i)
+__global__ void repack_gu(uint8_t* dst_layer0, size_t layer_stride, size_t off, const uint16_t* wg,
+                          const uint16_t* wu, Dims dm) {
+    const int r = blockIdx.x, l = blockIdx.y;
+    const uint16_t* src = ((r & 1) ? wu : wg) + ((size_t)l * dm.F + (r >> 1)) * dm.d;
+    const uint4* s = reinterpret_cast<const uint4*>(src);
+    uint4* d = reinterpret_cast<uint4*>(dst_layer0 + (size_t)l * layer_stride + off + (size_t)r * dm.d * 2);
+    for (int i = threadIdx.x; i < dm.d / 8; i += blockDim.x) d[i] = s[i];
+}
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15) == 0; }
+
+}  // namespace
+
+// ------------------------------------------------------------------ C ABI
+
+extern "C" {
+
+size_t kd_arena_bytes(const kd_config* cfg) {
+    if (!valid_config(cfg)) return 0;
+    return make_layout(make_dims(cfg)).total;
+}
+
+double kd_step_bytes(const kd_config* cfg, int64_t kv_positions, int with_head) {
+    if (!valid_config(cfg) || kv_positions < 0) return -1.0;
+    const double d = cfg->d_model, hd = cfg->head_dim, Hq = cfg->n_heads, Hkv = cfg->n_kv_heads;
+    const double F = cfg->ffn_dim, L = cfg->n_layers, V = cfg->vocab;
+    // per layer: two norm gains, Wq/Wk/Wv, Wo, gate/up, down
+    const double layer = 2 * d + (Hq + 2 * Hkv) * hd * d + Hq * hd * d + 2 * F * d + F * d;
+    double elems = L * layer + d;  // + the embedding row of the input token
+    if (with_head) elems += d + V * d;
+    const double kv = L * Hkv * (double)kv_positions * hd * 2;  // K and V rows
+    return 2.0 * (elems + kv);
+}
+
+int kd_create(const kd_config* cfg, void* d_arena, size_t arena_bytes, void* stream, kd_ctx** out) {
+    if (!out) return KD_EINVAL;
+    *out = nullptr;
+    if (!valid_config(cfg) || !d_arena) return KD_EINVAL;
+    kd_ctx* c = (kd_ctx*)calloc(1, sizeof(kd_ctx));
+    if (!c) return KD_EINVAL;
+    c->cfg = *cfg;
+    c->dm = make_dims(cfg);
+    c->lay = make_layout(c->dm);
+    c->arena = (uint8_t*)d_arena;
+    c->stream = (cudaStream_t)stream;
+    c->timeout_ns = 1000000000LL;
+    if (const char* t = getenv("KD_TIMEOUT_MS")) c->timeout_ns = atoll(t) * 1000000LL;
+    int rc = KD_OK;
+    if (arena_bytes < c->lay.total || ((uintptr_t)d_arena & 255)) {
+        rc = fail(c, KD_ENOMEM, "arena of %zu bytes at %p; need %zu bytes, 256-byte aligned", arena_bytes,
+                  d_arena, c->lay.total);
+    }
+    cudaDeviceProp prop;
+    if (rc == KD_OK) {
+        cudaError_t e = cudaGetDevice(&c->device);
+        if (e == cudaSuccess) e = cudaGetDeviceProperties(&prop, c->device);
+        if (e != cudaSuccess) rc = fail(c, KD_ECUDA, "device query failed: %s", cudaGetErrorString(e));
+    }
+    if (rc == KD_OK && !prop.cooperativeLaunch) rc = fail(c, KD_ECOOP, "device lacks cooperative launch");
+    if (rc == KD_OK) {
+        const Dims& d = c->dm;
+        c->nb = prop.multiProcessorCount;
+        if (c->nb > kMaxGrid) c->nb = kMaxGrid;
+        c->pieces = c->nb / d.Hkv;
+        c->pos_per_stage = kStageBytes / (2 * d.hd * 2);
+        int xs = d.d;
+        if (d.qd > xs) xs = d.qd;
+        if (d.F > xs) xs = d.F;
+        const int merge = kConsumerWarps * d.r * (d.hd + 2);
+        if (merge > xs) xs = merge;
+        c->xs_floats = (xs + 31) & ~31;
+        Params p{};
+        p.xs_floats = c->xs_floats;
+        p.ns = 1;
+        const int fixed = monokernel_smem_bytes(p) - kStageBytes;
+        c->ns = (kSmemLimit - fixed) / kStageBytes;
+        if (c->ns > kMaxStages) c->ns = kMaxStages;
+        if (c->ns < 2) rc = fail(c, KD_EINVAL, "activation buffers leave no room for a pipeline");
+        if (rc == KD_OK) {
+            p.ns = c->ns;
+            c->smem = monokernel_smem_bytes(p);
+            int per_sm = 0;
+            int e = monokernel_occupancy(c->smem, &per_sm);
+            if (e != 0) rc = fail(c, KD_ECUDA, "occupancy query failed: %s", cudaGetErrorString((cudaError_t)e));
+            else if (per_sm < 1)
+                rc = fail(c, KD_ECOOP, "monokernel cannot be resident (smem %d bytes)", c->smem);
+        }
+    }
+    if (rc == KD_OK) {
+        cudaError_t e = cudaMemsetAsync(c->arena + c->lay.ctl, 0, (size_t)kCtlWords * 8, c->stream);
+        if (e != cudaSuccess) rc = fail(c, KD_ECUDA, "cudaMemsetAsync: %s", cudaGetErrorString(e));
+    }
+    if (rc != KD_OK) {
+        fprintf(stderr, "kd_create: %s\n", c->err);
+        free(c);
+        return rc;
+    }
+    *out = c;
+    return KD_OK;
+}
+
+int kd_load_weights(kd_ctx* c, const kd_weights* w) {
+    if (!c || !w) return KD_EINVAL;
+    const void* ptrs[] = {w->embed, w->attn_norm, w->wq, w->wk, w->wv, w->wo, w->ffn_norm,
+                          w->wg, w->wu, w->wd, w->final_norm, w->lm_head};
+    for (const void* p : ptrs)
+        if (!p || !aligned16(p)) return fail(c, KD_EINVAL, "weight pointer NULL or not 16-byte aligned");
+    const Dims& d = c->dm;
+    const Layout& y = c->lay;
+    cudaStream_t s = c->stream;
+    const size_t D = d.d;
+    KD_CUDA(c, cudaMemcpyAsync(c->arena + y.embed, w->embed, (size_t)d.V * D * 2, cudaMemcpyDeviceToDevice, s));
+    KD_CUDA(c, cudaMemcpyAsync(c->arena + y.lm_head, w->lm_head, (size_t)d.V * D * 2, cudaMemcpyDeviceToDevice, s));
+    KD_CUDA(c, cudaMemcpyAsync(c->arena + y.final_norm, w->final_norm, D * 2, cudaMemcpyDeviceToDevice, s));
+    uint8_t* l0 = c->arena + y.layer0;
+    auto per_layer = [&](size_t off, const void* src, size_t bytes) {
+        return cudaMemcpy2DAsync(l0 + off, y.layer_stride, src, bytes, bytes, d.L, cudaMemcpyDeviceToDevice, s);
+    };
+    KD_CUDA(c, per_layer(y.l_attn_norm, w->attn_norm, D * 2));
+    KD_CUDA(c, per_layer(y.l_ffn_norm, w->ffn_norm, D * 2));
+    KD_CUDA(c, per_layer(y.l_wo, w->wo, D * d.qd * 2));
+    KD_CUDA(c, per_layer(y.l_wd, w->wd, D * d.F * 2));
+    repack_qkv<<<dim3(d.qkv_rows, d.L), 128, 0, s>>>(l0, y.layer_stride, y.l_wqkv, (const uint16_t*)w->wq,
+                                                      (const uint16_t*)w->wk, (const uint16_t*)w->wv, d);
+    KD_CUDA(c, cudaGetLastError());
+    repack_gu<<<dim3(2 * d.F, d.L), 128, 0, s>>>(l0, y.layer_stride, y.l_wgu, (const uint16_t*)w->wg,
+                                                  (const uint16_t*)w->wu, d);
+    KD_CUDA(c, cudaGetLastError());
+    c->launches += 2;
+    c->has_weights = true;
+    return KD_OK;
+}
+
+int kd_set_kv(kd_ctx* c, int32_t layer, int32_t which, const void* d_src, int32_t n_pos) {
+    if (!c || !d_src) return KD_EINVAL;
+    const Dims& d = c->dm;
+    if (layer < 0 || layer >= d.L || (which != 0 && which != 1) || n_pos < 0 || n_pos > d.S)
+        return fail(c, KD_EINVAL, "kd_set_kv: bad layer/which/n_pos");
+    if (n_pos == 0) return KD_OK;
+    uint8_t* dst = c->arena + (which ? c->lay.vcache : c->lay.kcache) + (size_t)layer * d.Hkv * d.S * d.hd * 2;
+    const size_t w = (size_t)n_pos * d.hd * 2;
+    KD_CUDA(c, cudaMemcpy2DAsync(dst, (size_t)d.S * d.hd * 2, d_src, w, w, d.Hkv, cudaMemcpyDeviceToDevice,
+                                 c->stream));
+    return KD_OK;
+}
+
+void* kd_kv_ptr(kd_ctx* c, int32_t layer, int32_t which) {
+    if (!c || layer < 0 || layer >= c->dm.L || (which != 0 && which != 1)) return nullptr;
+    return c->arena + (which ? c->lay.vcache : c->lay.kcache) + (size_t)layer * c->dm.Hkv * c->dm.S * c->dm.hd * 2;
+}
+
+static int reset_common(kd_ctx* c, int32_t n_tokens, int32_t kv_len) {
+    if (n_tokens < 1 || kv_len < 0 || kv_len >= c->dm.S || n_tokens > c->dm.S)
+        return fail(c, KD_EINVAL, "kd_reset: need n_tokens >= 1 and 0 <= kv_len < max_seq");
+    // Control words are left consistent by every completed launch (the kernel re-bases
+    // its barrier count and clears its own argmax slots), so they are cleared only after a
+    // failed run: the decode path then involves no memset.
+    if (c->failed) KD_CUDA(c, cudaMemsetAsync(c->arena + c->lay.ctl, 0, (size_t)kCtlWords * 8, c->stream));
+    c->pos = kv_len;
+    c->n_pending = n_tokens;
+    c->failed = false;
+    return KD_OK;
+}
+
+int kd_reset(kd_ctx* c, const int32_t* d_tokens, int32_t n_tokens, int32_t kv_len) {
+    if (!c || !d_tokens) return KD_EINVAL;
+    int rc = reset_common(c, n_tokens, kv_len);
+    if (rc) return rc;
+    KD_CUDA(c, cudaMemcpyAsync(c->arena + c->lay.tokens_in, d_tokens, (size_t)n_tokens * 4,
+                               cudaMemcpyDeviceToDevice, c->stream));
+    return KD_OK;
+}
+
+int kd_decode(kd_ctx* c, int32_t n_gen, int32_t* d_tokens_out, float* d_logits_out) {
+    if (!c) return KD_EINVAL;
+    if (!c->has_weights || c->n_pending < 1) return fail(c, KD_ESTATE, "kd_decode: no weights or nothing pending");
+    if (c->failed) return fail(c, KD_ESTATE, "kd_decode: an earlier run failed; call kd_reset");
+    if (n_gen < 0 || (n_gen > 0 && !d_tokens_out)) return fail(c, KD_EINVAL, "kd_decode: bad n_gen / tokens_out");
+    const int steps = c->n_pending + n_gen - 1;
+    if (steps == 0) return KD_OK;
+    if ((long long)c->pos + steps > c->dm.S)
+        return fail(c, KD_ECAPACITY, "kd_decode: position %d + %d steps exceeds max_seq %d", c->pos, steps, c->dm.S);
+    Params p{};
+    p.arena = c->arena;
+    p.lay = c->lay;
+    p.dm = c->dm;
+    p.steps = steps;
+    p.n_pending = c->n_pending;
+    p.pos0 = c->pos;
+    p.n_gen = n_gen;
+    p.dump = d_logits_out != nullptr;
+    p.tokens_out = d_tokens_out;
+    p.logits_out = d_logits_out;
+    p.nb = c->nb;
+    p.ns = c->ns;
+    p.attn_pieces = c->pieces;
+    p.pos_per_stage = c->pos_per_stage;
+    p.rows_qkv = rows_per_stage(c->dm.d, true);
+    p.rows_o = rows_per_stage(c->dm.qd, false);
+    p.rows_gu = rows_per_stage(c->dm.d, true);
+    p.rows_d = rows_per_stage(c->dm.F, false);
+    p.rows_lm = rows_per_stage(c->dm.d, false);
+    p.xs_floats = c->xs_floats;
+    p.timeout_ns = c->timeout_ns;
+    p.trace = c->trace;
+    p.trace_every = c->trace_every;
+    p.trace_rows = c->trace_rows;
+    int e = 0;
+    launch_decode(p, c->stream, c->smem, &e);
+    if (e != 0) return fail(c, KD_ECUDA, "cooperative launch failed: %s", cudaGetErrorString((cudaError_t)e));
+    c->launches += 1;
+    c->pos += steps;
+    c->n_pending = 1;
+    return KD_OK;
+}
+
+int kd_sync(kd_ctx* c) {
+    if (!c) return KD_EINVAL;
+    KD_CUDA(c, cudaStreamSynchronize(c->stream));
+    unsigned long long st[2] = {0, 0};
+    KD_CUDA(c, cudaMemcpyAsync(st, c->arena + c->lay.ctl + (size_t)kCtlStatus * 8, sizeof st,
+                               cudaMemcpyDeviceToHost, c->stream));
+    KD_CUDA(c, cudaStreamSynchronize(c->stream));
+    if (st[0] != 0) {
+        c->failed = true;
+        const unsigned w = (unsigned)st[1];
+        return fail(c, KD_ETIMEOUT, "device wait exceeded its limit (kind %u, cta %u, detail %u)", w >> 24,
+                    (w >> 8) & 0xffff, w & 0xff);
+    }
+    return KD_OK;
+}
+
+int kd_generate(kd_ctx* c, const int32_t* h_tokens, int32_t n_tokens, int32_t kv_len, int32_t n_gen,
+                int32_t* h_tokens_out) {
+    if (!c || !h_tokens || (n_gen > 0 && !h_tokens_out)) return KD_EINVAL;
+    int rc = reset_common(c, n_tokens, kv_len);
+    if (rc) return rc;
+    int32_t* d_tok_out = (int32_t*)(c->arena + c->lay.tokens_out);
+    KD_CUDA(c, cudaMemcpyAsync(c->arena + c->lay.tokens_in, h_tokens, (size_t)n_tokens * 4,
+                               cudaMemcpyHostToDevice, c->stream));
+    rc = kd_decode(c, n_gen, d_tok_out, nullptr);
+    if (rc) return rc;
+    if (n_gen > 0)
+        KD_CUDA(c, cudaMemcpyAsync(h_tokens_out, d_tok_out, (size_t)n_gen * 4, cudaMemcpyDeviceToHost, c->stream));
+    return kd_sync(c);
+}
+
+int kd_set_trace(kd_ctx* c, unsigned long long* d_buf, int64_t n_words, int32_t every) {
+    if (!c) return KD_EINVAL;
+    if (!d_buf) {
+        c->trace = nullptr;
+        return KD_OK;
+    }
+    if (every < 1) return fail(c, KD_EINVAL, "kd_set_trace: every must be >= 1");
+    const int64_t traced = (c->nb + every - 1) / every;
+    const int64_t rows = n_words / (traced * kTraceWords);
+    if (rows < 2 || rows > (1 << 30)) return fail(c, KD_EINVAL, "kd_set_trace: buffer too small");
+    c->trace = d_buf;
+    c->trace_every = every;
+    c->trace_rows = (int)rows;
+    return KD_OK;
+}
+
+int32_t kd_position(const kd_ctx* c) { return c ? c->pos : -1; }
+
+int kd_get_info(const kd_ctx* c, kd_info* info) {
+    if (!c || !info) return KD_EINVAL;
+    info->grid = c->nb;
+    info->threads = kThreads;
+    info->smem_bytes = c->smem;
+    info->stages = c->ns;
+    info->stage_bytes = kStageBytes;
+    info->attn_pieces = c->pieces;
+    info->arena_bytes = (int64_t)c->lay.total;
+    info->weight_bytes = (int64_t)c->lay.weights_end;
+    info->kv_bytes = (int64_t)c->lay.kv_bytes;
+    info->launches = c->launches;
+    return KD_OK;
+}
+
+const char* kd_last_error(const kd_ctx* c) { return c ? c->err : "no handle"; }
+
+const char* kd_strerror(int code) {
+    switch (code) {
+        case KD_OK: return "ok";
+        case KD_EINVAL: return "invalid argument or unsupported configuration";
+        case KD_ENOMEM: return "arena too small or misaligned";
+        case KD_ECAPACITY: return "KV capacity (max_seq) exceeded";
+        case KD_ECOOP: return "kernel cannot be co-resident on every SM";
+        case KD_ECUDA: return "CUDA runtime error";
+        case KD_ETIMEOUT: return "device-side wait exceeded its limit";
+        case KD_ESTATE: return "call out of order";
+        default: return "unknown error";
+    }
+}
+
+void kd_destroy(kd_ctx* c) { free(c); }
+
+}  // extern "C"

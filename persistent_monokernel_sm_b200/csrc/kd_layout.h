@@ -1,0 +1,95 @@
+// kd_layout.h -- arena layout, launch constants and kernel parameters shared by the host
+// side of libkd (kd_api.cu) and the monokernel (kd_kernel.cu). Internal to libkd.
+#pragma once
+
+#include <stddef.h>
+#include <stdint.h>
+
+namespace kd {
+
+// Pipeline: one producer warp streams weight / KV tiles into a ring of shared-memory
+// stages with 1-D bulk copies; consumer warps each take whole stages round-robin.
+constexpr int kStageBytes = 32768;
+constexpr int kConsumerWarps = 8;
+constexpr int kConsumerThreads = 32 * kConsumerWarps;
+constexpr int kThreads = kConsumerThreads + 32;
+constexpr int kMaxRows = 16;      // rows of one GEMV stage (register accumulators)
+constexpr int kMaxGroup = 8;      // q heads per kv head
+constexpr int kMaxKvHeads = 16;
+constexpr int kMaxStages = 8;
+constexpr int kSmemLimit = 232448;  // opt-in dynamic shared memory per CTA on B200
+static_assert(kMaxStages <= kConsumerWarps, "each ring slot needs its own consumer warp");
+
+// Control words (uint64), each on its own 128-byte line.
+constexpr int kCtlBar = 0;                 // grid-barrier arrivals, monotonic
+constexpr int kCtlStatus = 16;             // 0 = ok, else an error code (device side)
+constexpr int kCtlWhere = 17;              // where a wait gave up (debug)
+constexpr int kCtlArgmax = 32;             // 3 argmax slots at kCtlArgmax + 16*i
+constexpr int kCtlHead = 96;               // split-K arrival counters at kCtlHead + 16*g
+constexpr int kCtlWords = kCtlHead + 16 * kMaxKvHeads;
+
+constexpr int kStatusTimeout = 1;
+
+struct Dims {
+    int L, d, Hq, Hkv, hd, F, V, S;  // S = max_seq
+    float eps, theta;
+    int qd, kvd, r;  // Hq*hd, Hkv*hd, Hq/Hkv
+    int qkv_rows;    // (Hq + 2*Hkv) * hd
+};
+
+// Byte offsets inside the arena.
+struct Layout {
+    size_t embed, lm_head, final_norm;
+    size_t layer0, layer_stride;
+    size_t l_attn_norm, l_ffn_norm, l_wqkv, l_wo, l_wgu, l_wd;  // within a layer block
+    size_t kcache, vcache;                                        // [L][Hkv][S][hd] bf16
+    size_t x, q, o, hdn, part;                                    // fp32 scratch
+    size_t ctl, tokens_in, tokens_out;
+    size_t weights_end, kv_bytes, total;
+};
+
+// Rows per pipeline stage of one GEMV phase with reduction length K (bf16 elements);
+// `paired` phases keep row pairs (RoPE pairs, gate/up pairs) inside one stage.
+inline int rows_per_stage(int K, bool paired) {
+    int r = kStageBytes / (2 * K);
+    if (r > kMaxRows) r = kMaxRows;
+    if (paired) r &= ~1;
+    return r;
+}
+
+struct Params {
+    // weights (arena)
+    const uint8_t* arena;
+    Layout lay;
+    Dims dm;
+    // per-launch
+    int steps;      // decode steps in this launch
+    int n_pending;  // tokens fed before the first generated one
+    int pos0;       // position of step 0
+    int n_gen;
+    int dump;       // write logits of every step
+    int32_t* tokens_out;
+    float* logits_out;
+    // launch shape
+    int nb;           // CTAs
+    int ns;           // pipeline stages
+    int attn_pieces;  // CTAs per kv head in attention
+    int pos_per_stage;
+    int rows_qkv, rows_o, rows_gu, rows_d, rows_lm;  // rows per stage of each GEMV phase
+    int xs_floats;                                    // activation buffer (floats)
+    long long timeout_ns;
+    // optional trace: CTAs with blockIdx.x % trace_every == 0 record per-phase timestamps
+    unsigned long long* trace;
+    int trace_every, trace_rows;  // rows per traced CTA (4 words each)
+};
+
+// Trace row layout (SM clock cycles): consumer rows [begin, loaded, arrive, done] per phase,
+// in phase order; the last row of a traced CTA holds the producer's
+// [cycles blocked on a free slot, cycles blocked on a KV epoch, stages issued, total cycles].
+constexpr int kTraceWords = 4;
+
+void launch_decode(const Params& p, void* stream, int smem_bytes, int* err);
+int monokernel_smem_bytes(const Params& p);
+int monokernel_occupancy(int smem_bytes, int* blocks_per_sm);
+
+}  // namespace kd
