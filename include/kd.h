@@ -142,6 +142,25 @@ int kd_generate(kd_ctx *ctx, const int32_t *h_tokens, int32_t n_tokens, int32_t 
  * KD_ETIMEOUT) or a CUDA error. */
 int kd_sync(kd_ctx *ctx);
 
+/* kd_decode without device working memory of its own: the pages have no counterpart; this
+ * is a service to callers that cannot allocate device memory while decoding (for example an
+ * engine whose memory pool is fully committed at start-up and forbids cudaMalloc later, or
+ * a host that can only lend the library buffers it registered in advance).
+ * It resets the request like kd_reset (d_tokens: device int32 [n_tokens], the first at
+ * position kv_len) and generates n_gen tokens in one launch, exactly like kd_decode, but the
+ * activation vectors, attention partials, control words and pending tokens live in a 1 MiB
+ * array inside the library (loaded on every GPU that loads libkd, held until exit) instead of
+ * in the arena's scratch region. The weights and KV cache are still the handle's arena.
+ * Inputs and outputs as for kd_decode; calls KD_EINVAL with a message when this model and
+ * n_tokens need more than the 1 MiB. It calls no allocator: the control words are cleared
+ * with a memset and the tokens copied in, then it waits for the launch and returns its
+ * device status. The array keeps the last call's contents and every call shares it, so
+ * calls that overlap on the GPU (two streams, two handles) race: serialise them. The first
+ * call on a device looks the array's address up (cudaGetSymbolAddress), so make that first
+ * call outside any stream capture. The handle's position and pending tokens are not changed. */
+int kd_decode_noalloc(kd_ctx *ctx, const int32_t *d_tokens, int32_t n_tokens, int32_t kv_len,
+                      int32_t n_gen, int32_t *d_tokens_out, float *d_logits_out);
+
 /* Optional phase trace for performance analysis (off by default). While set, every
  * decode launch has each CTA with index % every == 0 record, per phase and in phase order,
  * four SM-clock stamps: phase begin, activation vector loaded, arrival at the grid

@@ -160,6 +160,25 @@ bool aligned16(const void* p) { return ((uintptr_t)p & 15) == 0; }
 
 }  // namespace
 
+// ------------------------------------------------------------------ internal accessors
+
+int kd_internal_view(kd_ctx* c, kd_ctx_view* v) {
+    if (!c || !v) return KD_EINVAL;
+    v->dm = &c->dm;
+    v->lay = &c->lay;
+    v->arena = c->arena;
+    v->stream = c->stream;
+    v->device = c->device, v->nb = c->nb, v->smem = c->smem, v->ns = c->ns;
+    v->pieces = c->pieces, v->pos_per_stage = c->pos_per_stage, v->xs_floats = c->xs_floats;
+    v->timeout_ns = c->timeout_ns;
+    v->has_weights = c->has_weights;
+    return KD_OK;
+}
+
+int kd_internal_fail(kd_ctx* c, int code, const char* msg) { return fail(c, code, "%s", msg); }
+
+void kd_internal_count_launch(kd_ctx* c) { c->launches += 1; }
+
 // ------------------------------------------------------------------ C ABI
 
 extern "C" {

@@ -89,6 +89,17 @@ struct Params {
 constexpr int kTraceWords = 4;
 
 void launch_decode(const Params& p, void* stream, int smem_bytes, int* err);
+
+// Read-only view of a handle's internals for entry points defined outside kd_api.cu.
+struct kd_ctx_view {
+    const Dims* dm;
+    const Layout* lay;
+    uint8_t* arena;
+    void* stream;
+    int device, nb, smem, ns, pieces, pos_per_stage, xs_floats;
+    long long timeout_ns;
+    bool has_weights;
+};
 int monokernel_smem_bytes(const Params& p);
 int monokernel_occupancy(int smem_bytes, int* blocks_per_sm);
 
