@@ -163,11 +163,13 @@ int kd_decode_noalloc(kd_ctx *ctx, const int32_t *d_tokens, int32_t n_tokens, in
 
 /* Optional phase trace for performance analysis (off by default). While set, every
  * decode launch has each CTA with index % every == 0 record, per phase and in phase order,
- * four SM-clock stamps: phase begin, activation vector loaded, arrival at the grid
- * barrier, barrier passed. Traced CTA i owns rows [i * R, (i + 1) * R) of the buffer, where
- * R = n_words / (4 * ceil(grid / every)); its last row holds the producer warp's cycles
- * blocked on a free pipeline stage, cycles blocked on a KV epoch, stages issued and total
- * cycles. d_buf: device memory of n_words uint64 (caller-owned); NULL turns tracing off. */
+ * a row of eight SM-clock stamps: phase begin, activation vector loaded, arrival at the grid
+ * barrier, barrier passed, then (attention phase only, else 0) q loaded, cache pieces done,
+ * partial record written, cross-CTA combine done. Traced CTA i owns rows [i * R, (i + 1) * R)
+ * of the buffer, where R = n_words / (8 * ceil(grid / every)); its last row holds the producer
+ * warp's cycles blocked on a free pipeline stage, cycles blocked on a KV epoch, stages issued
+ * and total cycles. d_buf: device memory of n_words uint64 (caller-owned); NULL turns
+ * tracing off. */
 int kd_set_trace(kd_ctx *ctx, unsigned long long *d_buf, int64_t n_words, int32_t every);
 
 /* Next KV position to be written (host-side view, valid once calls were enqueued). */

@@ -98,6 +98,7 @@ struct kd_ctx {
     int pos, n_pending;
     long long launches;
     long long timeout_ns;
+    int prefetch;
     unsigned long long* trace;
     int trace_every, trace_rows;
     char err[512];
@@ -171,6 +172,7 @@ int kd_internal_view(kd_ctx* c, kd_ctx_view* v) {
     v->device = c->device, v->nb = c->nb, v->smem = c->smem, v->ns = c->ns;
     v->pieces = c->pieces, v->pos_per_stage = c->pos_per_stage, v->xs_floats = c->xs_floats;
     v->timeout_ns = c->timeout_ns;
+    v->prefetch = c->prefetch;
     v->has_weights = c->has_weights;
     return KD_OK;
 }
@@ -213,6 +215,8 @@ int kd_create(const kd_config* cfg, void* d_arena, size_t arena_bytes, void* str
     c->stream = (cudaStream_t)stream;
     c->timeout_ns = 1000000000LL;
     if (const char* t = getenv("KD_TIMEOUT_MS")) c->timeout_ns = atoll(t) * 1000000LL;
+    c->prefetch = 6;
+    if (const char* t = getenv("KD_PREFETCH")) c->prefetch = atoi(t);
     int rc = KD_OK;
     if (arena_bytes < c->lay.total || ((uintptr_t)d_arena & 255)) {
         rc = fail(c, KD_ENOMEM, "arena of %zu bytes at %p; need %zu bytes, 256-byte aligned", arena_bytes,
@@ -230,12 +234,14 @@ int kd_create(const kd_config* cfg, void* d_arena, size_t arena_bytes, void* str
         c->nb = prop.multiProcessorCount;
         if (c->nb > kMaxGrid) c->nb = kMaxGrid;
         c->pieces = c->nb / d.Hkv;
-        c->pos_per_stage = kStageBytes / (2 * d.hd * 2);
+        // attention stages: 8 positions per consumer warp (16 for hd 64), K then V rows
+        c->pos_per_stage = (d.hd == 128 ? 8 : 16) * kConsumerWarps;
         int xs = d.d;
         if (d.qd > xs) xs = d.qd;
         if (d.F > xs) xs = d.F;
         const int merge = kConsumerWarps * d.r * (d.hd + 2);
         if (merge > xs) xs = merge;
+        if (kMaxGroup * c->pieces + kMaxGroup > xs) xs = kMaxGroup * c->pieces + kMaxGroup;  // combine weights
         c->xs_floats = (xs + 31) & ~31;
         Params p{};
         p.xs_floats = c->xs_floats;
@@ -370,6 +376,7 @@ int kd_decode(kd_ctx* c, int32_t n_gen, int32_t* d_tokens_out, float* d_logits_o
     p.rows_lm = rows_per_stage(c->dm.d, false);
     p.xs_floats = c->xs_floats;
     p.timeout_ns = c->timeout_ns;
+    p.prefetch = c->prefetch;
     p.trace = c->trace;
     p.trace_every = c->trace_every;
     p.trace_rows = c->trace_rows;

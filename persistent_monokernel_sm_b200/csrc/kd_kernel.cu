@@ -6,13 +6,13 @@
 // prefetch and execution order).
 //
 // B200 design (one CTA per SM, 148 CTAs):
-//  * Warp specialisation. Warp 8 of each CTA is the producer: one lane walks the CTA's
+//  * Warp specialisation. Warp 7 of each CTA is the producer: one lane walks the CTA's
 //    fixed schedule of weight tiles (and KV-cache tiles) and streams them HBM -> shared
 //    memory with 1-D bulk async copies (cp.async.bulk) into a ring of 32 KB stages guarded
-//    by mbarriers. Warps 0-7 are consumers; ring slot i belongs to consumer warp i, which
-//    takes each stage that lands there whole. (A parity wait on an mbarrier can only tell
-//    the current phase from the one before it, so the warp that waits on a slot must be
-//    the one that finished the slot's previous stage.)
+//    by mbarriers. Warps 0-6 are consumers; every consumer warp takes part in every stage
+//    in order (a parity wait on an mbarrier can only tell the current phase from the one
+//    before it, so a warp must have finished a slot's previous stage before it waits on
+//    the slot again). 256 threads per CTA leave each thread the full 255 registers.
 //  * Weights never depend on activations, so the producer keeps streaming while the
 //    consumers wait at a grid barrier: the ring absorbs barrier latency instead of leaving
 //    HBM idle (the pages name prefetch and synchronisation control as the monokernel's
@@ -128,10 +128,15 @@ __device__ __forceinline__ int where_code(int what, int detail) {
 struct Tracer {
     unsigned long long* row0 = nullptr;
     int row = 0, rows = 0;
+    unsigned long long waited = 0;  // cycles thread 0 spent on full-stage waits this phase
     __device__ void mark(int col) {
         if (row0 && row < rows - 1) row0[(size_t)row * kTraceWords + col] = (unsigned long long)clock64();
     }
-    __device__ void next() { ++row; }
+    __device__ void next() {
+        if (row0 && row < rows - 1) row0[(size_t)row * kTraceWords + 6] = waited;
+        waited = 0;
+        ++row;
+    }
 };
 
 // ------------------------------------------------------------------ schedule geometry
@@ -214,42 +219,56 @@ struct Smem {
     int* flag;              // broadcast slots
     uint64_t* full;         // mbarriers
     uint64_t* empty;
-    float* sp;              // per-stage partial sums [slot][phase][row * KS + slice] (16 each)
-    int* scnt;              // per-stage arrival counts [slot][phase]
+    float* sp;              // per-stage partial sums [slot][row][warp]
+    int* scnt;              // per-stage arrival counts [slot]
 };
 
-__device__ __forceinline__ Smem carve(const Params& P, uint8_t* base) {
-    Smem s;
+// Byte offsets of the shared-memory regions; each starts on a 128-byte boundary (vector
+// loads and bulk-copy destinations need 16). Used by the kernel and for the launch size.
+struct SmemLayout {
+    size_t ring, xs, qs, rope, red, best, flag, full, empty, sp, scnt, total;
+};
+__host__ __device__ inline SmemLayout smem_layout(int ns, int xs_floats) {
+    SmemLayout L;
     size_t off = 0;
-    s.ring = base;
-    off += (size_t)P.ns * kStageBytes;
-    s.xs = reinterpret_cast<float*>(base + off);
-    off += (size_t)P.xs_floats * 4;
-    s.qs = reinterpret_cast<float*>(base + off);
-    off += (size_t)kMaxGroup * 128 * 4;
-    s.rope = reinterpret_cast<float2*>(base + off);
-    off += 64 * 8;
-    s.red = reinterpret_cast<float*>(base + off);
-    off += 64 * 4;
-    s.best = reinterpret_cast<unsigned long long*>(base + off);
-    off += kConsumerWarps * 8;
-    s.flag = reinterpret_cast<int*>(base + off);
-    off += 16 * 4;
-    s.full = reinterpret_cast<uint64_t*>(base + off);
-    off += kMaxStages * 8;
-    s.empty = reinterpret_cast<uint64_t*>(base + off);
-    off += kMaxStages * 8;
-    s.sp = reinterpret_cast<float*>(base + off);
-    off += (size_t)kMaxStages * 2 * kMaxRows * 4;
-    s.scnt = reinterpret_cast<int*>(base + off);
+    auto take = [&](size_t bytes) {
+        const size_t at = off;
+        off = (off + bytes + 127) & ~(size_t)127;
+        return at;
+    };
+    L.ring = take((size_t)ns * kStageBytes);
+    L.xs = take((size_t)xs_floats * 4);
+    L.qs = take((size_t)kMaxGroup * 128 * 4);
+    L.rope = take(64 * 8);
+    L.red = take(64 * 4);
+    L.best = take((size_t)kConsumerWarps * 8);
+    L.flag = take(16 * 4);
+    L.full = take((size_t)kMaxStages * 8);
+    L.empty = take((size_t)kMaxStages * 8);
+    L.sp = take((size_t)kMaxStages * kMaxRows * 8 * 4);
+    L.scnt = take((size_t)kMaxStages * 4);
+    L.total = off;
+    return L;
+}
+
+__device__ __forceinline__ Smem carve(const Params& P, uint8_t* base) {
+    const SmemLayout L = smem_layout(P.ns, P.xs_floats);
+    Smem s;
+    s.ring = base + L.ring;
+    s.xs = reinterpret_cast<float*>(base + L.xs);
+    s.qs = reinterpret_cast<float*>(base + L.qs);
+    s.rope = reinterpret_cast<float2*>(base + L.rope);
+    s.red = reinterpret_cast<float*>(base + L.red);
+    s.best = reinterpret_cast<unsigned long long*>(base + L.best);
+    s.flag = reinterpret_cast<int*>(base + L.flag);
+    s.full = reinterpret_cast<uint64_t*>(base + L.full);
+    s.empty = reinterpret_cast<uint64_t*>(base + L.empty);
+    s.sp = reinterpret_cast<float*>(base + L.sp);
+    s.scnt = reinterpret_cast<int*>(base + L.scnt);
     return s;
 }
 
-int monokernel_smem_bytes(const Params& p) {
-    return p.ns * kStageBytes + p.xs_floats * 4 + kMaxGroup * 128 * 4 + 64 * 8 + 64 * 4 +
-           kConsumerWarps * 8 + 16 * 4 + 2 * kMaxStages * 8 + kMaxStages * 2 * kMaxRows * 4 +
-           kMaxStages * 2 * 4;
-}
+int monokernel_smem_bytes(const Params& p) { return (int)smem_layout(p.ns, p.xs_floats).total; }
 
 // Split layout of an activation vector of length K (K % 8 == 0): element k lives at
 // ((k & 7) >> 2) * (K / 2) + (k >> 3) * 4 + (k & 3), so lane-strided 8-element chunks
@@ -285,12 +304,20 @@ __device__ __forceinline__ bool mbar_wait_hint(uint32_t a, uint32_t parity) {
     return ok != 0;
 }
 
-__device__ bool wait_full(const Smem& sm, const Ring& rg, const Params& P, unsigned long long* ctl) {
+__device__ bool wait_full(const Smem& sm, const Ring& rg, const Params& P, unsigned long long* ctl,
+                          unsigned long long* waited = nullptr) {
     const uint32_t a = smem_u32(&sm.full[rg.slot]);
-    if (__all_sync(0xffffffffu, mbar_try_wait(a, rg.phase))) return true;
+    const long long c0 = clock64();
+    if (__all_sync(0xffffffffu, mbar_try_wait(a, rg.phase))) {
+        if (waited) *waited += (unsigned long long)(clock64() - c0);
+        return true;
+    }
     const uint64_t t0 = globaltimer();
     for (;;) {
-        if (__all_sync(0xffffffffu, mbar_wait_hint(a, rg.phase))) return true;
+        if (__all_sync(0xffffffffu, mbar_wait_hint(a, rg.phase))) {
+            if (waited) *waited += (unsigned long long)(clock64() - c0);
+            return true;
+        }
         int bad = 0;
         if ((threadIdx.x & 31) == 0) {
             bad = read_status(ctl) != 0;
@@ -408,161 +435,266 @@ struct StepCtx {
     unsigned long long lm_best;  // running argmax key of this warp (lane 0)
 };
 
-// Partial dot products of one warp's share of a stage: rows [ra, ra + nr) (nr <= 2) over
-// the 8-element chunks [c0, c1) of the row, lane-strided; returns the warp-reduced sums.
-__device__ __forceinline__ void gemv_part(const uint8_t* st, size_t rowb, int ra, int nr, int c0, int c1,
-                                          const float* xs, int K, float& s0, float& s1) {
+// Sum N values per lane across the 32 lanes with log-depth exchanges that halve the
+// number of live values at each step: afterwards lane (i << (5 - log2 N)) holds the total
+// of value i (N = 1, 2, 4 or 8; 5, 5, 6 or 9 shuffles). Compile-time recursion keeps every
+// index static, so the values stay in registers.
+template <int N, int BIT>
+__device__ __forceinline__ float multi_reduce_step(const float (&v)[N], int lane) {
+    if constexpr (N == 1) {
+        float x = v[0];
+#pragma unroll
+        for (int o = BIT; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+        return x;
+    } else {
+        constexpr int H = N / 2;
+        const bool upper = (lane & BIT) != 0;
+        float w[H];
+#pragma unroll
+        for (int i = 0; i < H; ++i) {
+            // keep the half selected by this lane's bit, send the other half to the partner
+            const float send = upper ? v[i] : v[i + H];
+            const float keep = upper ? v[i + H] : v[i];
+            w[i] = keep + __shfl_xor_sync(0xffffffffu, send, BIT);
+        }
+        return multi_reduce_step<H, BIT / 2>(w, lane);
+    }
+}
+template <int N>
+__device__ __forceinline__ float multi_reduce(const float (&v)[N]) {
+    return multi_reduce_step<N, 16>(v, threadIdx.x & 31);
+}
+
+// One warp's share of a GEMV stage: all n (<= RMAX) rows of the stage over the 8-element
+// chunks [c0, c1) of the reduction dimension, lane-strided. Each activation chunk is read
+// once and used for every row (RMAX independent accumulators). Leaves this lane's partial
+// sum of each row in v[] (reduce across lanes with multi_reduce).
+template <int RMAX>
+__device__ __forceinline__ void gemv_part(const uint8_t* st, size_t rowb, int n, int c0, int c1, const float* xs,
+                                          int K, float (&v)[RMAX]) {
     const int lane = threadIdx.x & 31;
-    float a0 = 0.f, b0 = 0.f, a1 = 0.f, b1 = 0.f;
+    constexpr int SUB = RMAX >= 4 ? 1 : 4 / RMAX;  // accumulators per row (latency hiding)
+    float acc[RMAX][SUB];
+#pragma unroll
+    for (int r = 0; r < RMAX; ++r)
+#pragma unroll
+        for (int u = 0; u < SUB; ++u) acc[r][u] = 0.f;
     const float4* xlo = reinterpret_cast<const float4*>(xs);
     const float4* xhi = reinterpret_cast<const float4*>(xs + (K >> 1));
-    const uint8_t* w0 = st + (size_t)ra * rowb;
-    const uint8_t* w1 = w0 + rowb;
-    if (nr == 2) {
-#pragma unroll 4
-        for (int c = c0 + lane; c < c1; c += 32) {
-            const float4 x = xlo[c], y = xhi[c];
-            const uint4 p = *reinterpret_cast<const uint4*>(w0 + (size_t)c * 16);
-            const uint4 q = *reinterpret_cast<const uint4*>(w1 + (size_t)c * 16);
-            a0 = fmaf(bf_lo(p.x), x.x, a0); b0 = fmaf(bf_hi(p.x), x.y, b0);
-            a0 = fmaf(bf_lo(p.y), x.z, a0); b0 = fmaf(bf_hi(p.y), x.w, b0);
-            a0 = fmaf(bf_lo(p.z), y.x, a0); b0 = fmaf(bf_hi(p.z), y.y, b0);
-            a0 = fmaf(bf_lo(p.w), y.z, a0); b0 = fmaf(bf_hi(p.w), y.w, b0);
-            a1 = fmaf(bf_lo(q.x), x.x, a1); b1 = fmaf(bf_hi(q.x), x.y, b1);
-            a1 = fmaf(bf_lo(q.y), x.z, a1); b1 = fmaf(bf_hi(q.y), x.w, b1);
-            a1 = fmaf(bf_lo(q.z), y.x, a1); b1 = fmaf(bf_hi(q.z), y.y, b1);
-            a1 = fmaf(bf_lo(q.w), y.z, a1); b1 = fmaf(bf_hi(q.w), y.w, b1);
-        }
-    } else if (nr == 1) {
-#pragma unroll 4
-        for (int c = c0 + lane; c < c1; c += 32) {
-            const float4 x = xlo[c], y = xhi[c];
-            const uint4 p = *reinterpret_cast<const uint4*>(w0 + (size_t)c * 16);
-            a0 = fmaf(bf_lo(p.x), x.x, a0); b0 = fmaf(bf_hi(p.x), x.y, b0);
-            a0 = fmaf(bf_lo(p.y), x.z, a0); b0 = fmaf(bf_hi(p.y), x.w, b0);
-            a0 = fmaf(bf_lo(p.z), y.x, a0); b0 = fmaf(bf_hi(p.z), y.y, b0);
-            a0 = fmaf(bf_lo(p.w), y.z, a0); b0 = fmaf(bf_hi(p.w), y.w, b0);
+#pragma unroll 2
+    for (int c = c0 + lane; c < c1; c += 32) {
+        const float4 x = xlo[c], y = xhi[c];
+#pragma unroll
+        for (int r = 0; r < RMAX; ++r) {
+            if (r < n) {
+                const uint4 w = *reinterpret_cast<const uint4*>(st + r * rowb + (size_t)c * 16);
+                const float f[8] = {bf_lo(w.x), bf_hi(w.x), bf_lo(w.y), bf_hi(w.y),
+                                    bf_lo(w.z), bf_hi(w.z), bf_lo(w.w), bf_hi(w.w)};
+                const float g[8] = {x.x, x.y, x.z, x.w, y.x, y.y, y.z, y.w};
+#pragma unroll
+                for (int e = 0; e < 8; ++e) acc[r][e % SUB] = fmaf(f[e], g[e], acc[r][e % SUB]);
+            }
         }
     }
-    s0 = a0 + b0;
-    s1 = a1 + b1;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        s0 += __shfl_xor_sync(0xffffffffu, s0, o);
-        s1 += __shfl_xor_sync(0xffffffffu, s1, o);
+    for (int r = 0; r < RMAX; ++r) {
+        float t = acc[r][0];
+#pragma unroll
+        for (int u = 1; u < SUB; ++u) t += acc[r][u];
+        v[r] = t;
     }
 }
 
-// One GEMV phase. Every consumer warp takes part in every stage: the stage's R rows are
-// split into RG row groups x KS column slices (RG * KS = 8 warps, at most 2 rows per
-// warp), each warp writes its partial sums to shared memory, and the last warp to finish
-// the stage adds the KS slices in a fixed order and applies the phase's epilogue.
+// Phase epilogue for the rows [r0, r0 + n) of one stage; lane i holds row r0 + i's total.
+__device__ __forceinline__ void gemv_epilogue(const Params& P, const Smem& sm, int phase, int l, int r0, int n,
+                                              float tot, StepCtx& sc, float* xg) {
+    const Dims& dm = P.dm;
+    const int lane = threadIdx.x & 31;
+    if (phase == kQKV || phase == kGU) {
+        const float nb = __shfl_down_sync(0xffffffffu, tot, 1);
+        if (!(lane & 1) && lane < n) {
+            const float a = tot, b = nb;
+            const int row = r0 + lane;  // even row of a (RoPE pair | gate, up) pair
+            if (phase == kGU) {
+                float* hdn = reinterpret_cast<float*>(const_cast<uint8_t*>(P.arena) + P.lay.hdn);
+                __stcg(hdn + (row >> 1), a / (1.0f + expf(-a)) * b);
+            } else if (row < dm.qd + dm.kvd) {
+                const int hd = dm.hd;
+                const bool isq = row < dm.qd;
+                const int rr = isq ? row : row - dm.qd;
+                const int h = rr / hd, i = (rr % hd) >> 1;
+                const float2 cs = sm.rope[i];
+                const float ra_ = a * cs.x - b * cs.y;
+                const float rb_ = b * cs.x + a * cs.y;
+                if (isq) {
+                    float* q = reinterpret_cast<float*>(const_cast<uint8_t*>(P.arena) + P.lay.q);
+                    __stcg(q + h * hd + i, ra_);
+                    __stcg(q + h * hd + i + hd / 2, rb_);
+                } else {
+                    __nv_bfloat16* kc = reinterpret_cast<__nv_bfloat16*>(const_cast<uint8_t*>(P.arena) + P.lay.kcache) +
+                                        (((size_t)l * dm.Hkv + h) * dm.S + sc.p) * hd;
+                    kc[i] = __float2bfloat16_rn(ra_);
+                    kc[i + hd / 2] = __float2bfloat16_rn(rb_);
+                    fence_proxy_async_global();
+                }
+            } else {
+                const int rr = row - dm.qd - dm.kvd;
+                const int h = rr / dm.hd, j2 = rr % dm.hd;
+                __nv_bfloat16* vc = reinterpret_cast<__nv_bfloat16*>(const_cast<uint8_t*>(P.arena) + P.lay.vcache) +
+                                    (((size_t)l * dm.Hkv + h) * dm.S + sc.p) * dm.hd;
+                vc[j2] = __float2bfloat16_rn(a);
+                vc[j2 + 1] = __float2bfloat16_rn(b);
+                fence_proxy_async_global();
+            }
+        }
+    } else if (phase == kO || phase == kD) {
+        if (lane < n) __stcg(xg + r0 + lane, __ldcg(xg + r0 + lane) + tot);
+    } else {  // LM head: dump, then this warp's running argmax (lowest index on ties)
+        if (P.dump && lane < n) __stcg(P.logits_out + (size_t)sc.t * dm.V + r0 + lane, tot);
+        unsigned long long key = lane < n ? argmax_key(tot, r0 + lane) : 0ull;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const unsigned long long other = __shfl_xor_sync(0xffffffffu, key, o);
+            key = other > key ? other : key;
+        }
+        if (lane == 0 && key > sc.lm_best) sc.lm_best = key;
+    }
+}
+
+// One GEMV phase. Every consumer warp takes part in every stage: warp w reduces all R rows
+// of the stage over the w-th seventh of the reduction dimension and writes its R partial
+// sums to shared memory; the last warp to finish the stage adds the seven slices in a fixed
+// order, releases the stage, and applies the phase's epilogue to the R rows.
 // A wait that gives up marks `ok` false and the warp skips the work of the remaining
 // stages, but it still reaches every named barrier; the next grid barrier then reports
 // the failure to the whole CTA at once.
-__device__ void run_gemv(const Params& P, const Smem& sm, unsigned long long* ctl, int phase, int l,
-                         Ring& rg, StepCtx& sc, bool& ok) {
+template <int RMAX>
+__device__ __noinline__ void run_gemv_t(const Params& P, const Smem& sm_ref, unsigned long long* ctl, int phase, int l,
+                                       const Gemv& g_ref, Ring& rg_ref, StepCtx& sc_ref, bool& ok_ref, Tracer& tr) {
+    // This is a separate function (its own register allocation); work on register copies of
+    // the caller's state and write back at the end.
+    const Smem sm = sm_ref;
+    const Gemv g = g_ref;
+    Ring rg = rg_ref;
+    StepCtx sc = sc_ref;
+    bool ok = ok_ref;
+    constexpr int SHIFT = RMAX == 8 ? 2 : RMAX == 4 ? 3 : RMAX == 2 ? 4 : 5;
     const Dims& dm = P.dm;
-    const Gemv g = gemv_geom(P, phase, l, blockIdx.x);
     const int nst = gemv_stages(g);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int RG = g.R >= 8 ? 8 : (g.R >= 4 ? 4 : (g.R >= 2 ? 2 : 1));
-    const int KS = kConsumerWarps / RG;
-    const int grp = warp / KS, ks = warp % KS;
     const int nch = g.K >> 3;
-    const int c0 = nch * ks / KS, c1 = nch * (ks + 1) / KS;
+    const int c0 = nch * warp / kConsumerWarps, c1 = nch * (warp + 1) / kConsumerWarps;
     const size_t rowb = (size_t)g.K * 2;
     float* xg = reinterpret_cast<float*>(const_cast<uint8_t*>(P.arena) + P.lay.x);
-    for (int j = 0; j < nst; ++j, rg.advance(P.ns)) {
-        if (!ok) continue;
-        if (!wait_full(sm, rg, P, ctl)) {
-            ok = false;
+    unsigned long long* waited = threadIdx.x == 0 ? &tr.waited : nullptr;
+    // Two stages in flight per warp: the loads and FMAs of stage j + 1 are issued before the
+    // cross-lane reduction and epilogue of stage j, hiding the latter's latency.
+    float cur[RMAX], nxt[RMAX];
+    Ring rj = rg;  // ring position of stage j
+    if (nst > 0 && ok) {
+        if (!wait_full(sm, rj, P, ctl, waited)) ok = false;
+        else gemv_part<RMAX>(sm.ring + (size_t)rj.slot * kStageBytes, rowb, min(g.R, g.row1 - g.row0), c0, c1, sm.xs,
+                             g.K, cur);
+    }
+    for (int j = 0; j < nst; ++j) {
+        Ring rn = rj;
+        rn.advance(P.ns);
+        if (!ok) {
+            rj = rn;
             continue;
+        }
+        if (j + 1 < nst) {
+            if (!wait_full(sm, rn, P, ctl, waited)) {
+                ok = false;
+                rj = rn;
+                continue;
+            }
+            const int rn0 = g.row0 + (j + 1) * g.R;
+            gemv_part<RMAX>(sm.ring + (size_t)rn.slot * kStageBytes, rowb, min(g.R, g.row1 - rn0), c0, c1, sm.xs, g.K,
+                            nxt);
         }
         const int r0 = g.row0 + j * g.R;
         const int n = min(g.R, g.row1 - r0);
-        const int ra = n * grp / RG, nr = n * (grp + 1) / RG - ra;
-        float s0, s1;
-        gemv_part(sm.ring + (size_t)rg.slot * kStageBytes, rowb, ra, nr, c0, c1, sm.xs, g.K, s0, s1);
+        const float part = multi_reduce<RMAX>(cur);
+        float* sp = sm.sp + (size_t)rj.slot * (kMaxRows * 8);  // [row][warp], rows padded to 8 warps
+        const int prow = lane >> SHIFT;
+        if ((lane & ((1 << SHIFT) - 1)) == 0 && prow < n) sp[prow * 8 + warp] = part;
         __syncwarp();
-        // rows * KS <= kMaxRows for every split (R >= 8 -> KS = 1; R < 8 -> R * KS < 16)
-        float* sp = sm.sp + (size_t)(rg.slot * 2 + rg.phase) * kMaxRows;
-        int* cnt = sm.scnt + rg.slot * 2 + rg.phase;
         int last = 0;
         if (lane == 0) {
-            mbar_arrive(smem_u32(&sm.empty[rg.slot]));  // this warp is done reading the stage
-            if (nr > 0) sp[ra * KS + ks] = s0;
-            if (nr > 1) sp[(ra + 1) * KS + ks] = s1;
             __threadfence_block();
-            last = atomicAdd(cnt, 1) == kConsumerWarps - 1;
+            last = atomicAdd(&sm.scnt[rj.slot], 1) == kConsumerWarps - 1;
+            if (!last) mbar_arrive(smem_u32(&sm.empty[rj.slot]));  // done with the stage
         }
-        if (!__shfl_sync(0xffffffffu, last, 0)) continue;
-        // ---- last warp of this stage: row totals (lane = row) and the epilogue
-        __threadfence_block();
-        float tot = 0.f;
-        if (lane < n)
-            for (int q = 0; q < KS; ++q) tot += sp[lane * KS + q];
-        if (lane == 0) *cnt = 0;
-        if (phase == kQKV || phase == kGU) {
-            const float nb = __shfl_down_sync(0xffffffffu, tot, 1);
-            if (!(lane & 1) && lane < n) {
-                const float a = tot, b = nb;
-                const int row = r0 + lane;  // even row of a (RoPE pair | gate, up) pair
-                if (phase == kGU) {
-                    float* hdn = reinterpret_cast<float*>(const_cast<uint8_t*>(P.arena) + P.lay.hdn);
-                    __stcg(hdn + (row >> 1), a / (1.0f + expf(-a)) * b);
-                } else if (row < dm.qd + dm.kvd) {
-                    const int hd = dm.hd;
-                    const bool isq = row < dm.qd;
-                    const int rr = isq ? row : row - dm.qd;
-                    const int h = rr / hd, i = (rr % hd) >> 1;
-                    const float2 cs = sm.rope[i];
-                    const float ra_ = a * cs.x - b * cs.y;
-                    const float rb_ = b * cs.x + a * cs.y;
-                    if (isq) {
-                        float* q = reinterpret_cast<float*>(const_cast<uint8_t*>(P.arena) + P.lay.q);
-                        __stcg(q + h * hd + i, ra_);
-                        __stcg(q + h * hd + i + hd / 2, rb_);
-                    } else {
-                        __nv_bfloat16* kc = reinterpret_cast<__nv_bfloat16*>(const_cast<uint8_t*>(P.arena) + P.lay.kcache) +
-                                            (((size_t)l * dm.Hkv + h) * dm.S + sc.p) * hd;
-                        kc[i] = __float2bfloat16_rn(ra_);
-                        kc[i + hd / 2] = __float2bfloat16_rn(rb_);
-                        fence_proxy_async_global();
-                    }
-                } else {
-                    const int rr = row - dm.qd - dm.kvd;
-                    const int h = rr / dm.hd, j2 = rr % dm.hd;
-                    __nv_bfloat16* vc = reinterpret_cast<__nv_bfloat16*>(const_cast<uint8_t*>(P.arena) + P.lay.vcache) +
-                                        (((size_t)l * dm.Hkv + h) * dm.S + sc.p) * dm.hd;
-                    vc[j2] = __float2bfloat16_rn(a);
-                    vc[j2 + 1] = __float2bfloat16_rn(b);
-                    fence_proxy_async_global();
-                }
+        if (__shfl_sync(0xffffffffu, last, 0)) {
+            // ---- last warp of this stage: row totals (lane = row), release, epilogue
+            __threadfence_block();
+            float tot = 0.f;
+            if (lane < n) {
+                const float4 a = *reinterpret_cast<const float4*>(sp + lane * 8);
+                const float4 b = *reinterpret_cast<const float4*>(sp + lane * 8 + 4);
+                static_assert(kConsumerWarps == 7, "row totals add 7 warp slices");
+                tot = ((a.x + a.y) + (a.z + a.w)) + ((b.x + b.y) + b.z);
             }
-        } else if (phase == kO || phase == kD) {
-            if (lane < n) __stcg(xg + r0 + lane, __ldcg(xg + r0 + lane) + tot);
-        } else {  // LM head: dump, then this warp's running argmax (lowest index on ties)
-            if (P.dump && lane < n) __stcg(P.logits_out + (size_t)sc.t * dm.V + r0 + lane, tot);
-            unsigned long long key = lane < n ? argmax_key(tot, r0 + lane) : 0ull;
+            __syncwarp();
+            if (lane == 0) {
+                sm.scnt[rj.slot] = 0;
+                mbar_arrive(smem_u32(&sm.empty[rj.slot]));  // partial sums read: the slot may refill
+            }
+            gemv_epilogue(P, sm, phase, l, r0, n, tot, sc, xg);
+        }
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                const unsigned long long other = __shfl_xor_sync(0xffffffffu, key, o);
-                key = other > key ? other : key;
-            }
-            if (lane == 0 && key > sc.lm_best) sc.lm_best = key;
-        }
+        for (int r = 0; r < RMAX; ++r) cur[r] = nxt[r];
+        rj = rn;
+    }
+    rg_ref = rj;
+    sc_ref.lm_best = sc.lm_best;
+    ok_ref = ok;
+}
+
+__device__ void run_gemv(const Params& P, const Smem& sm, unsigned long long* ctl, int phase, int l, Ring& rg,
+                         StepCtx& sc, bool& ok, Tracer& tr) {
+    const Gemv g = gemv_geom(P, phase, l, blockIdx.x);
+    if (g.R <= 1) run_gemv_t<1>(P, sm, ctl, phase, l, g, rg, sc, ok, tr);
+    else if (g.R <= 2) run_gemv_t<2>(P, sm, ctl, phase, l, g, rg, sc, ok, tr);
+    else if (g.R <= 4) run_gemv_t<4>(P, sm, ctl, phase, l, g, rg, sc, ok, tr);
+    else run_gemv_t<8>(P, sm, ctl, phase, l, g, rg, sc, ok, tr);  // rows_per_stage caps R at 8
+}
+
+// Loads that read either the shared-memory ring or, for the current position, the cache
+// itself (written during this launch: L2 only).
+__device__ __forceinline__ uint4 ld16(const __nv_bfloat16* p, bool global) {
+    return global ? __ldcg(reinterpret_cast<const uint4*>(p)) : *reinterpret_cast<const uint4*>(p);
+}
+template <int E>
+__device__ __forceinline__ void ld_v(const __nv_bfloat16* p, bool global, float (&v)[E]) {
+    if constexpr (E == 4) {
+        const uint2 w = global ? __ldcg(reinterpret_cast<const uint2*>(p)) : *reinterpret_cast<const uint2*>(p);
+        v[0] = bf_lo(w.x), v[1] = bf_hi(w.x), v[2] = bf_lo(w.y), v[3] = bf_hi(w.y);
+    } else {
+        const uint32_t w = global ? __ldcg(reinterpret_cast<const unsigned int*>(p)) : *reinterpret_cast<const uint32_t*>(p);
+        v[0] = bf_lo(w), v[1] = bf_hi(w);
     }
 }
 
-// ------------------------------------------------------------------ attention phase
-
-template <int HD>
-__device__ void run_attention(const Params& P, const Smem& sm, unsigned long long* ctl, int l, Ring& rg,
-                              StepCtx& sc, bool& ok) {
-    constexpr int E = HD / 32;  // dims per lane
+// Split-K decode attention for one kv head over this CTA's piece of the cache. Each warp
+// handles 8 positions per pass: lanes 4j..4j+3 hold position j's score (each lane a quarter
+// of the head dimension, q broadcast from shared memory), one max / rescale per pass, then
+// all lanes accumulate the 8 V rows (each lane hd/32 output dims). States of the warps are
+// merged per CTA; the last CTA of a kv head to finish combines all pieces.
+// GMAX >= the number of q heads per kv head (2, 4 or 8).
+template <int HD, int GMAX>
+__device__ __noinline__ void run_attention(const Params& P, const Smem& sm_ref, unsigned long long* ctl, int l,
+                                          Ring& rg_ref, StepCtx& sc_ref, bool& ok_ref, Tracer& tr) {
+    const Smem sm = sm_ref;  // register copies (see run_gemv_t)
+    const StepCtx sc = sc_ref;
+    Ring rg = rg_ref;
+    bool ok = ok_ref;
+    constexpr int CPL = HD / 32;  // 16-byte K chunks per lane (4 lanes per position)
+    constexpr int E = HD / 32;    // output dims per lane
     const Dims& dm = P.dm;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
+    const int pj = lane >> 2, qq = lane & 3;
     const Attn at = attn_geom(P, sc.p, blockIdx.x);
     if (at.g < 0) return;  // uniform across the CTA
     const int r = dm.r, A = P.attn_pieces;
@@ -570,91 +702,165 @@ __device__ void run_attention(const Params& P, const Smem& sm, unsigned long lon
     const float* qg = reinterpret_cast<const float*>(P.arena + P.lay.q) + (size_t)at.g * r * HD;
     for (int i = tid; i < r * HD; i += kConsumerThreads) sm.qs[i] = __ldcg(qg + i) * qscale;
     consumer_sync();
+    if (tid == 0) tr.mark(4);
 
-    float q[kMaxGroup][E], m[kMaxGroup], lsum[kMaxGroup], acc[kMaxGroup][E];
+    float m[GMAX], lsum[GMAX], acc[GMAX][E];
 #pragma unroll
-    for (int h = 0; h < kMaxGroup; ++h) {
+    for (int h = 0; h < GMAX; ++h) {
         m[h] = -INFINITY;
         lsum[h] = 0.f;
 #pragma unroll
-        for (int e = 0; e < E; ++e) {
-            acc[h][e] = 0.f;
-            q[h][e] = h < r ? sm.qs[h * HD + lane * E + e] : 0.f;
-        }
+        for (int e = 0; e < E; ++e) acc[h][e] = 0.f;
     }
-    auto visit = [&](const __nv_bfloat16* krow, const __nv_bfloat16* vrow, bool global) {
-        float kv[E], vv[E];
-        if constexpr (E == 4) {
-            uint2 kw, vw;
-            if (global) {
-                kw = __ldcg(reinterpret_cast<const uint2*>(krow + lane * E));
-                vw = __ldcg(reinterpret_cast<const uint2*>(vrow + lane * E));
-            } else {
-                kw = *reinterpret_cast<const uint2*>(krow + lane * E);
-                vw = *reinterpret_cast<const uint2*>(vrow + lane * E);
+    // One pass over two blocks of up to 8 positions each (A: rows at ka / va, B: rows at
+    // kb / vb): lanes 4j..4j+3 score position j of both blocks, then all lanes fold the up
+    // to 16 V rows into their output dims with a single rescale.
+    auto pass2 = [&](const __nv_bfloat16* ka, const __nv_bfloat16* va, int na, const __nv_bfloat16* kb,
+                     const __nv_bfloat16* vb, int nb, bool global) {
+        const bool ma = pj < na, mb = pj < nb;
+        float sa[GMAX][2], sb[GMAX][2];
+#pragma unroll
+        for (int h = 0; h < GMAX; ++h) sa[h][0] = sa[h][1] = sb[h][0] = sb[h][1] = 0.f;
+#pragma unroll
+        for (int i = 0; i < CPL; ++i) {
+            const int c = qq + 4 * i;
+            const uint4 wa = ma ? ld16(ka + (size_t)pj * HD + c * 8, global) : make_uint4(0, 0, 0, 0);
+            const uint4 wb = mb ? ld16(kb + (size_t)pj * HD + c * 8, global) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+            for (int h = 0; h < GMAX; ++h) {
+                if (h < r) {
+                    const float4 qa = *reinterpret_cast<const float4*>(&sm.qs[h * HD + c * 8]);
+                    const float4 qb = *reinterpret_cast<const float4*>(&sm.qs[h * HD + c * 8 + 4]);
+                    float t = sa[h][i & 1], u = sb[h][i & 1];
+                    t = fmaf(qa.x, bf_lo(wa.x), t); u = fmaf(qa.x, bf_lo(wb.x), u);
+                    t = fmaf(qa.y, bf_hi(wa.x), t); u = fmaf(qa.y, bf_hi(wb.x), u);
+                    t = fmaf(qa.z, bf_lo(wa.y), t); u = fmaf(qa.z, bf_lo(wb.y), u);
+                    t = fmaf(qa.w, bf_hi(wa.y), t); u = fmaf(qa.w, bf_hi(wb.y), u);
+                    t = fmaf(qb.x, bf_lo(wa.z), t); u = fmaf(qb.x, bf_lo(wb.z), u);
+                    t = fmaf(qb.y, bf_hi(wa.z), t); u = fmaf(qb.y, bf_hi(wb.z), u);
+                    t = fmaf(qb.z, bf_lo(wa.w), t); u = fmaf(qb.z, bf_lo(wb.w), u);
+                    t = fmaf(qb.w, bf_hi(wa.w), t); u = fmaf(qb.w, bf_hi(wb.w), u);
+                    sa[h][i & 1] = t;
+                    sb[h][i & 1] = u;
+                }
             }
-            kv[0] = bf_lo(kw.x), kv[1] = bf_hi(kw.x), kv[2] = bf_lo(kw.y), kv[3] = bf_hi(kw.y);
-            vv[0] = bf_lo(vw.x), vv[1] = bf_hi(vw.x), vv[2] = bf_lo(vw.y), vv[3] = bf_hi(vw.y);
-        } else {
-            uint32_t kw, vw;
-            if (global) {
-                kw = __ldcg(reinterpret_cast<const unsigned int*>(krow + lane * E));
-                vw = __ldcg(reinterpret_cast<const unsigned int*>(vrow + lane * E));
-            } else {
-                kw = *reinterpret_cast<const uint32_t*>(krow + lane * E);
-                vw = *reinterpret_cast<const uint32_t*>(vrow + lane * E);
+        }
+        float pa[GMAX], pb[GMAX];
+#pragma unroll
+        for (int h = 0; h < GMAX; ++h) {
+            pa[h] = pb[h] = 0.f;
+            if (h < r) {
+                float s0 = sa[h][0] + sa[h][1], s1 = sb[h][0] + sb[h][1];
+                s0 += __shfl_xor_sync(0xffffffffu, s0, 1);
+                s1 += __shfl_xor_sync(0xffffffffu, s1, 1);
+                s0 += __shfl_xor_sync(0xffffffffu, s0, 2);
+                s1 += __shfl_xor_sync(0xffffffffu, s1, 2);
+                if (!ma) s0 = -INFINITY;
+                if (!mb) s1 = -INFINITY;
+                float mx = fmaxf(s0, s1);
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+                const float mn = fmaxf(m[h], mx);  // finite: na >= 1
+                const float corr = exp2f(m[h] - mn);
+                const float e0 = exp2f(s0 - mn), e1 = exp2f(s1 - mn);
+                float ps = e0 + e1;
+                ps += __shfl_xor_sync(0xffffffffu, ps, 4);
+                ps += __shfl_xor_sync(0xffffffffu, ps, 8);
+                ps += __shfl_xor_sync(0xffffffffu, ps, 16);
+                lsum[h] = fmaf(lsum[h], corr, ps);
+#pragma unroll
+                for (int e = 0; e < E; ++e) acc[h][e] *= corr;
+                m[h] = mn;
+                pa[h] = e0;
+                pb[h] = e1;
             }
-            kv[0] = bf_lo(kw), kv[1] = bf_hi(kw);
-            vv[0] = bf_lo(vw), vv[1] = bf_hi(vw);
         }
 #pragma unroll
-        for (int h = 0; h < kMaxGroup; ++h) {
-            if (h < r) {
-                float s = 0.f;
+        for (int jj = 0; jj < 8; ++jj) {
+            float v0[E], v1[E];
+            if (jj < na) ld_v<E>(va + (size_t)jj * HD + lane * E, global, v0);
+            if (jj < nb) ld_v<E>(vb + (size_t)jj * HD + lane * E, global, v1);
 #pragma unroll
-                for (int e = 0; e < E; ++e) s = fmaf(q[h][e], kv[e], s);
+            for (int h = 0; h < GMAX; ++h) {
+                if (h < r) {
+                    const float p0 = __shfl_sync(0xffffffffu, pa[h], jj * 4);
+                    const float p1 = __shfl_sync(0xffffffffu, pb[h], jj * 4);
 #pragma unroll
-                for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-                const float mn = fmaxf(m[h], s);
-                const float corr = exp2f(m[h] - mn);
-                const float pr = exp2f(s - mn);
-                lsum[h] = lsum[h] * corr + pr;
-#pragma unroll
-                for (int e = 0; e < E; ++e) acc[h][e] = fmaf(acc[h][e], corr, pr * vv[e]);
-                m[h] = mn;
+                    for (int e = 0; e < E; ++e) {
+                        if (jj < na) acc[h][e] = fmaf(p0, v0[e], acc[h][e]);
+                        if (jj < nb) acc[h][e] = fmaf(p1, v1[e], acc[h][e]);
+                    }
+                }
             }
         }
     };
 
-    // every warp takes an eighth of each stage's positions and keeps its own softmax state
+    // This warp's positions of each stage: [n * w / W, n * (w + 1) / W) of the stage's n.
+    // With hd 128 that is at most 8, and two consecutive stages share one pass; with hd 64
+    // it is at most 16, split over one pass.
     const int nst = attn_stages(P, at);
-    for (int j = 0; j < nst; ++j, rg.advance(P.ns)) {
-        if (!ok) continue;
-        if (!wait_full(sm, rg, P, ctl)) {
+    unsigned long long* waited = tid == 0 ? &tr.waited : nullptr;
+    for (int j = 0; j < nst && ok;) {
+        if (!wait_full(sm, rg, P, ctl, waited)) {
             ok = false;
-            continue;
+            break;
         }
         const int s0 = at.a + j * P.pos_per_stage;
         const int n = min(P.pos_per_stage, at.tma_end - s0);
         const __nv_bfloat16* st = reinterpret_cast<const __nv_bfloat16*>(sm.ring + (size_t)rg.slot * kStageBytes);
-        const __nv_bfloat16* vst = st + (size_t)n * HD;
         const int p0 = n * warp / kConsumerWarps, p1 = n * (warp + 1) / kConsumerWarps;
-        for (int jj = p0; jj < p1; ++jj) visit(st + (size_t)jj * HD, vst + (size_t)jj * HD, false);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&sm.empty[rg.slot]));
+        const __nv_bfloat16* ka = st + (size_t)p0 * HD;
+        const __nv_bfloat16* va = st + (size_t)(n + p0) * HD;
+        const int na = min(8, p1 - p0);
+        Ring r2 = rg;
+        r2.advance(P.ns);
+        if (p1 - p0 > 8) {  // hd 64: both blocks from this stage
+            pass2(ka, va, na, ka + (size_t)8 * HD, va + (size_t)8 * HD, p1 - p0 - 8, false);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&sm.empty[rg.slot]));
+            rg = r2;
+            j += 1;
+        } else if (j + 1 < nst) {  // pair with the next stage
+            if (!wait_full(sm, r2, P, ctl, waited)) {
+                ok = false;
+                break;
+            }
+            const int s1 = at.a + (j + 1) * P.pos_per_stage;
+            const int n1 = min(P.pos_per_stage, at.tma_end - s1);
+            const __nv_bfloat16* st1 = reinterpret_cast<const __nv_bfloat16*>(sm.ring + (size_t)r2.slot * kStageBytes);
+            const int q0 = n1 * warp / kConsumerWarps, q1 = n1 * (warp + 1) / kConsumerWarps;
+            if (na > 0) pass2(ka, va, na, st1 + (size_t)q0 * HD, st1 + (size_t)(n1 + q0) * HD, q1 - q0, false);
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(smem_u32(&sm.empty[rg.slot]));
+                mbar_arrive(smem_u32(&sm.empty[r2.slot]));
+            }
+            r2.advance(P.ns);
+            rg = r2;
+            j += 2;
+        } else {
+            if (na > 0) pass2(ka, va, na, ka, va, 0, false);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&sm.empty[rg.slot]));
+            rg = r2;
+            j += 1;
+        }
     }
     // the current position, written by this step's QKV phase, read straight from the cache
     if (at.b > sc.p && warp == kConsumerWarps - 1) {
         const size_t off = (((size_t)l * dm.Hkv + at.g) * dm.S + sc.p) * HD;
-        visit(reinterpret_cast<const __nv_bfloat16*>(P.arena + P.lay.kcache) + off,
-              reinterpret_cast<const __nv_bfloat16*>(P.arena + P.lay.vcache) + off, true);
+        const __nv_bfloat16* kp = reinterpret_cast<const __nv_bfloat16*>(P.arena + P.lay.kcache) + off;
+        const __nv_bfloat16* vp = reinterpret_cast<const __nv_bfloat16*>(P.arena + P.lay.vcache) + off;
+        pass2(kp, vp, 1, kp, vp, 0, true);
     }
 
     // merge the warps' states (xs is free during attention)
+    if (tid == 0) tr.mark(5);
     const int rec = HD + 2;
     float* ws = sm.xs;  // [warp][h][rec]
 #pragma unroll
-    for (int h = 0; h < kMaxGroup; ++h) {
+    for (int h = 0; h < GMAX; ++h) {
         if (h < r) {
             float* wr = ws + ((size_t)warp * r + h) * rec;
             if (lane == 0) wr[0] = m[h], wr[1] = lsum[h];
@@ -692,35 +898,137 @@ __device__ void run_attention(const Params& P, const Smem& sm, unsigned long lon
     }
     consumer_sync();
     if (sm.flag[1]) {  // last piece of this kv head to finish: combine all pieces
-        float* og = reinterpret_cast<float*>(const_cast<uint8_t*>(P.arena) + P.lay.o) + (size_t)at.g * r * HD;
         const float* hp = part + (size_t)at.g * A * r * rec;
-        for (int idx = tid; idx < r * HD; idx += kConsumerThreads) {
-            const int h = idx / HD, dd = idx % HD;
+        float* fw = sm.xs;                    // [h][A] piece weights
+        float* invl = sm.xs + kMaxGroup * A;  // [h]
+        if (warp < r) {  // warp h: the weights 2^(m_i - M) of head h's pieces and 1 / L
+            const int h = warp;
             float M = -INFINITY;
-            for (int i = 0; i < A; ++i) M = fmaxf(M, __ldcg(hp + ((size_t)i * r + h) * rec));
-            float L = 0.f, o = 0.f;
-            for (int i = 0; i < A; ++i) {
+            for (int i = lane; i < A; i += 32) M = fmaxf(M, __ldcg(hp + ((size_t)i * r + h) * rec));
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+            float L = 0.f;
+            for (int i = lane; i < A; i += 32) {
                 const float* pr = hp + ((size_t)i * r + h) * rec;
                 const float mi = __ldcg(pr);
-                if (mi == -INFINITY) continue;
-                const float f = exp2f(mi - M);
+                const float f = mi == -INFINITY ? 0.f : exp2f(mi - M);
+                fw[h * A + i] = f;
                 L = fmaf(__ldcg(pr + 1), f, L);
-                o = fmaf(__ldcg(pr + 2 + dd), f, o);
             }
-            __stcg(og + (size_t)h * HD + dd, o / L);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+            if (lane == 0) invl[h] = 1.0f / L;
         }
+        consumer_sync();
+        float* og = reinterpret_cast<float*>(const_cast<uint8_t*>(P.arena) + P.lay.o) + (size_t)at.g * r * HD;
+        for (int idx = tid; idx < r * HD; idx += kConsumerThreads) {
+            const int h = idx / HD, dd = idx % HD;
+            const float* src = hp + (size_t)h * rec + 2 + dd;
+            const size_t stride = (size_t)r * rec;
+            float o0 = 0.f, o1 = 0.f, o2 = 0.f, o3 = 0.f;
+            int i = 0;
+            for (; i + 4 <= A; i += 4) {  // four independent loads in flight
+                const float a0 = __ldcg(src + (size_t)i * stride), a1 = __ldcg(src + (size_t)(i + 1) * stride);
+                const float a2 = __ldcg(src + (size_t)(i + 2) * stride), a3 = __ldcg(src + (size_t)(i + 3) * stride);
+                o0 = fmaf(a0, fw[h * A + i], o0);
+                o1 = fmaf(a1, fw[h * A + i + 1], o1);
+                o2 = fmaf(a2, fw[h * A + i + 2], o2);
+                o3 = fmaf(a3, fw[h * A + i + 3], o3);
+            }
+            for (; i < A; ++i) o0 = fmaf(__ldcg(src + (size_t)i * stride), fw[h * A + i], o0);
+            __stcg(og + (size_t)h * HD + dd, ((o0 + o1) + (o2 + o3)) * invl[h]);
+        }
+        if (tid == 0) tr.mark(7);
     }
+    rg_ref = rg;
+    ok_ref = ok;
 }
 
 // ------------------------------------------------------------------ producer
 
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
+// Walks this CTA's stages in consumption order: steps, layers, phases, stages.
+struct Cursor {
+    int t = 0, l = 0, ph = 0, j = 0, nst = 0;
+    bool done = false;
+    Gemv g;
+    Attn at;
+
+    __device__ void begin(const Params& P) {
+        done = P.steps <= 0;
+        if (!done) enter(P);
+        settle(P);
+    }
+    __device__ void enter(const Params& P) {
+        j = 0;
+        if (ph == kATT) {
+            at = attn_geom(P, P.pos0 + t, blockIdx.x);
+            nst = at.g < 0 ? 0 : attn_stages(P, at);
+        } else {
+            g = gemv_geom(P, ph, ph == kLM ? 0 : l, blockIdx.x);
+            nst = gemv_stages(g);
+        }
+    }
+    __device__ void settle(const Params& P) {
+        while (!done && j >= nst) {
+            if (ph < kD) {
+                ++ph;
+            } else if (ph == kD && l + 1 < P.dm.L) {
+                ++l;
+                ph = kQKV;
+            } else if (ph == kD && step_has_head(P, t)) {
+                ph = kLM;
+            } else {
+                ++t;
+                l = 0;
+                ph = kQKV;
+                if (t >= P.steps) {
+                    done = true;
+                    return;
+                }
+            }
+            enter(P);
+        }
+    }
+    __device__ void next(const Params& P) {
+        ++j;
+        settle(P);
+    }
+    // Source ranges of the current stage; kv_last >= 0 is the last cache position it reads.
+    __device__ void stage(const Params& P, const void*& s1, uint32_t& b1, const void*& s2, uint32_t& b2,
+                          int& kv_last) const {
+        if (ph == kATT) {
+            const Dims& dm = P.dm;
+            const int s0 = at.a + j * P.pos_per_stage;
+            const int n = min(P.pos_per_stage, at.tma_end - s0);
+            const size_t row = (((size_t)l * dm.Hkv + at.g) * dm.S + s0) * dm.hd;
+            s1 = reinterpret_cast<const __nv_bfloat16*>(P.arena + P.lay.kcache) + row;
+            s2 = reinterpret_cast<const __nv_bfloat16*>(P.arena + P.lay.vcache) + row;
+            b1 = b2 = (uint32_t)((size_t)n * dm.hd * 2);
+            kv_last = s0 + n - 1;
+        } else {
+            const size_t rowb = (size_t)g.K * 2;
+            const int r0 = g.row0 + j * g.R;
+            const int n = min(g.R, g.row1 - r0);
+            s1 = g.base + (size_t)r0 * rowb;
+            b1 = (uint32_t)(n * rowb);
+            s2 = nullptr;
+            b2 = 0;
+            kv_last = -1;
+        }
+    }
+};
+
 struct Producer {
     const Params& P;
-    const Smem& sm;
+    const Smem sm;
     unsigned long long* ctl;
     uint64_t base;
     uint64_t policy;
-    int k = 0;              // stages issued
+    int k = 0;               // stages issued
     int slot = 0, pass = 0;  // ring position of stage k: slot k % ns, pass k / ns
     long long seen_epochs = 0;
     unsigned long long wait_slot = 0, wait_kv = 0;  // cycles blocked (trace)
@@ -772,13 +1080,21 @@ struct Producer {
         return true;
     }
 
-    __device__ bool issue(const void* src, uint32_t bytes, const void* src2, uint32_t bytes2) {
+    __device__ bool issue(const Cursor& cur) {
+        const void *s1, *s2;
+        uint32_t b1, b2;
+        int kv_last;
+        cur.stage(P, s1, b1, s2, b2, kv_last);
+        if (kv_last >= P.pos0) {  // written earlier in this launch: wait for its QKV barrier
+            const long long need = barriers_before_step(P, kv_last - P.pos0) + 5ll * cur.l + 1;
+            if (!wait_epochs(need)) return false;
+        }
         if (!wait_empty()) return false;
         const uint32_t fb = smem_u32(&sm.full[slot]);
         const uint32_t dst = smem_u32(sm.ring + (size_t)slot * kStageBytes);
-        mbar_expect_tx(fb, bytes + bytes2);
-        bulk_g2s(dst, src, bytes, fb, policy);
-        if (bytes2) bulk_g2s(dst + bytes, src2, bytes2, fb, policy);
+        mbar_expect_tx(fb, b1 + b2);
+        bulk_g2s(dst, s1, b1, fb, policy);
+        if (b2) bulk_g2s(dst + b1, s2, b2, fb, policy);
         ++k;
         if (++slot == P.ns) {
             slot = 0;
@@ -787,45 +1103,31 @@ struct Producer {
         return true;
     }
 
-    __device__ bool gemv(int phase, int l) {
-        const Gemv g = gemv_geom(P, phase, l, blockIdx.x);
-        const size_t rowb = (size_t)g.K * 2;
-        for (int r0 = g.row0; r0 < g.row1; r0 += g.R) {
-            const int n = min(g.R, g.row1 - r0);
-            if (!issue(g.base + (size_t)r0 * rowb, (uint32_t)(n * rowb), nullptr, 0)) return false;
-        }
-        return true;
-    }
-
-    __device__ bool attention(int t, int l) {
-        const int p = P.pos0 + t;
-        const Attn at = attn_geom(P, p, blockIdx.x);
-        if (at.g < 0) return true;
-        const Dims& dm = P.dm;
-        const size_t head = ((size_t)l * dm.Hkv + at.g) * dm.S;
-        const __nv_bfloat16* kc = reinterpret_cast<const __nv_bfloat16*>(P.arena + P.lay.kcache);
-        const __nv_bfloat16* vc = reinterpret_cast<const __nv_bfloat16*>(P.arena + P.lay.vcache);
-        for (int s0 = at.a; s0 < at.tma_end; s0 += P.pos_per_stage) {
-            const int n = min(P.pos_per_stage, at.tma_end - s0);
-            const int last = s0 + n - 1;
-            if (last >= P.pos0) {  // written earlier in this launch: wait for its QKV barrier
-                const long long need = barriers_before_step(P, last - P.pos0) + 5ll * l + 1;
-                if (!wait_epochs(need)) return false;
-            }
-            const uint32_t bytes = (uint32_t)((size_t)n * dm.hd * 2);
-            if (!issue(kc + (head + s0) * dm.hd, bytes, vc + (head + s0) * dm.hd, bytes)) return false;
-        }
-        return true;
+    // Pull a later stage's bytes into L2 ahead of time; no shared memory, no completion to
+    // track, and harmless if a line is written afterwards (L2 is the coherence point).
+    __device__ void prefetch(const Cursor& cur) {
+        const void *s1, *s2;
+        uint32_t b1, b2;
+        int kv_last;
+        cur.stage(P, s1, b1, s2, b2, kv_last);
+        bulk_prefetch_l2(s1, b1);
+        if (b2) bulk_prefetch_l2(s2, b2);
     }
 
     __device__ void run() {
         const long long c_start = clock64();
         bool ok = true;
-        for (int t = 0; t < P.steps && ok; ++t) {
-            for (int l = 0; l < P.dm.L && ok; ++l) {
-                ok = gemv(kQKV, l) && attention(t, l) && gemv(kO, l) && gemv(kGU, l) && gemv(kD, l);
+        Cursor ld, pf;
+        ld.begin(P);
+        pf.begin(P);
+        for (int i = 0; i < P.prefetch && !pf.done; ++i, pf.next(P)) prefetch(pf);
+        while (ok && !ld.done) {
+            if (!pf.done) {
+                prefetch(pf);
+                pf.next(P);
             }
-            if (ok && step_has_head(P, t)) ok = gemv(kLM, 0);
+            ok = issue(ld);
+            ld.next(P);
         }
         if (!ok) {
             // unwinding: let every copy already issued land before the CTA exits
@@ -859,7 +1161,7 @@ __global__ void __launch_bounds__(kThreads, 1) monokernel(const __grid_constant_
         for (int s = 0; s < P.ns; ++s) {
             mbar_init(smem_u32(&sm.full[s]), 1);
             mbar_init(smem_u32(&sm.empty[s]), kConsumerWarps);  // every consumer warp releases
-            sm.scnt[2 * s] = sm.scnt[2 * s + 1] = 0;
+            sm.scnt[s] = 0;
         }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         // Barrier count at launch: a multiple of nb plus arrivals of CTAs that already
@@ -934,24 +1236,31 @@ __global__ void __launch_bounds__(kThreads, 1) monokernel(const __grid_constant_
             if (l == 0) load_rmsnorm(sm, nullptr, erow, gattn, dm.d, dm.eps);
             else load_rmsnorm(sm, xg, nullptr, gattn, dm.d, dm.eps);
             if (tid == 0) tr.mark(1);
-            run_gemv(P, sm, ctl, kQKV, l, rg, sc, ok);
+            run_gemv(P, sm, ctl, kQKV, l, rg, sc, ok, tr);
             if (!(ok = grid_sync(sm, epoch, base, P, ctl, ok, tr))) break;
             if (tid == 0) tr.mark(1);
-            if (dm.hd == 128) run_attention<128>(P, sm, ctl, l, rg, sc, ok);
-            else run_attention<64>(P, sm, ctl, l, rg, sc, ok);
+            if (dm.hd == 128) {
+                if (dm.r <= 2) run_attention<128, 2>(P, sm, ctl, l, rg, sc, ok, tr);
+                else if (dm.r <= 4) run_attention<128, 4>(P, sm, ctl, l, rg, sc, ok, tr);
+                else run_attention<128, 8>(P, sm, ctl, l, rg, sc, ok, tr);
+            } else {
+                if (dm.r <= 2) run_attention<64, 2>(P, sm, ctl, l, rg, sc, ok, tr);
+                else if (dm.r <= 4) run_attention<64, 4>(P, sm, ctl, l, rg, sc, ok, tr);
+                else run_attention<64, 8>(P, sm, ctl, l, rg, sc, ok, tr);
+            }
             if (!(ok = grid_sync(sm, epoch, base, P, ctl, ok, tr))) break;
             load_vector(sm, reinterpret_cast<const float*>(P.arena + P.lay.o), dm.qd);
             if (tid == 0) tr.mark(1);
-            run_gemv(P, sm, ctl, kO, l, rg, sc, ok);
+            run_gemv(P, sm, ctl, kO, l, rg, sc, ok, tr);
             if (!(ok = grid_sync(sm, epoch, base, P, ctl, ok, tr))) break;
             // feed-forward block
             load_rmsnorm(sm, xg, nullptr, gffn, dm.d, dm.eps);
             if (tid == 0) tr.mark(1);
-            run_gemv(P, sm, ctl, kGU, l, rg, sc, ok);
+            run_gemv(P, sm, ctl, kGU, l, rg, sc, ok, tr);
             if (!(ok = grid_sync(sm, epoch, base, P, ctl, ok, tr))) break;
             load_vector(sm, reinterpret_cast<const float*>(P.arena + P.lay.hdn), dm.F);
             if (tid == 0) tr.mark(1);
-            run_gemv(P, sm, ctl, kD, l, rg, sc, ok);
+            run_gemv(P, sm, ctl, kD, l, rg, sc, ok, tr);
             if (!(ok = grid_sync(sm, epoch, base, P, ctl, ok, tr))) break;
         }
         if (!ok) break;
@@ -959,7 +1268,7 @@ __global__ void __launch_bounds__(kThreads, 1) monokernel(const __grid_constant_
             load_rmsnorm(sm, xg, nullptr, reinterpret_cast<const __nv_bfloat16*>(P.arena + P.lay.final_norm),
                          dm.d, dm.eps);
             if (tid == 0) tr.mark(1);
-            run_gemv(P, sm, ctl, kLM, 0, rg, sc, ok);
+            run_gemv(P, sm, ctl, kLM, 0, rg, sc, ok, tr);
             if ((tid & 31) == 0) sm.best[tid >> 5] = sc.lm_best;
             consumer_sync();
             if (tid == 0 && ok) {

@@ -10,15 +10,14 @@ namespace kd {
 // Pipeline: one producer warp streams weight / KV tiles into a ring of shared-memory
 // stages with 1-D bulk copies; consumer warps each take whole stages round-robin.
 constexpr int kStageBytes = 32768;
-constexpr int kConsumerWarps = 8;
+constexpr int kConsumerWarps = 7;  // + 1 producer warp = 256 threads: the full register file
 constexpr int kConsumerThreads = 32 * kConsumerWarps;
 constexpr int kThreads = kConsumerThreads + 32;
-constexpr int kMaxRows = 16;      // rows of one GEMV stage (register accumulators)
+constexpr int kMaxRows = 8;       // rows of one GEMV stage (register accumulators)
 constexpr int kMaxGroup = 8;      // q heads per kv head
 constexpr int kMaxKvHeads = 16;
 constexpr int kMaxStages = 8;
 constexpr int kSmemLimit = 232448;  // opt-in dynamic shared memory per CTA on B200
-static_assert(kMaxStages <= kConsumerWarps, "each ring slot needs its own consumer warp");
 
 // Control words (uint64), each on its own 128-byte line.
 constexpr int kCtlBar = 0;                 // grid-barrier arrivals, monotonic
@@ -78,15 +77,18 @@ struct Params {
     int rows_qkv, rows_o, rows_gu, rows_d, rows_lm;  // rows per stage of each GEMV phase
     int xs_floats;                                    // activation buffer (floats)
     long long timeout_ns;
+    int prefetch;  // stages the producer pulls into L2 ahead of the shared-memory ring
     // optional trace: CTAs with blockIdx.x % trace_every == 0 record per-phase timestamps
     unsigned long long* trace;
     int trace_every, trace_rows;  // rows per traced CTA (4 words each)
 };
 
-// Trace row layout (SM clock cycles): consumer rows [begin, loaded, arrive, done] per phase,
-// in phase order; the last row of a traced CTA holds the producer's
-// [cycles blocked on a free slot, cycles blocked on a KV epoch, stages issued, total cycles].
-constexpr int kTraceWords = 4;
+// Trace row layout (SM clock cycles): consumer rows [begin, loaded, arrive, done, s4..s7] per
+// phase, in phase order, where s4..s7 are attention sub-steps (q loaded, cache pieces done,
+// partial record written, combine done; 0 elsewhere); the last row of a traced CTA holds the
+// producer's [cycles blocked on a free slot, cycles blocked on a KV epoch, stages issued,
+// total cycles].
+constexpr int kTraceWords = 8;
 
 void launch_decode(const Params& p, void* stream, int smem_bytes, int* err);
 
@@ -98,6 +100,7 @@ struct kd_ctx_view {
     void* stream;
     int device, nb, smem, ns, pieces, pos_per_stage, xs_floats;
     long long timeout_ns;
+    int prefetch;
     bool has_weights;
 };
 int monokernel_smem_bytes(const Params& p);

@@ -127,6 +127,7 @@ extern "C" int kd_decode_noalloc(kd_ctx* ctx, const int32_t* d_tokens, int32_t n
     p.rows_lm = rows_per_stage(dm.d, false);
     p.xs_floats = v.xs_floats;
     p.timeout_ns = v.timeout_ns;
+    p.prefetch = v.prefetch;
     int err = 0;
     launch_decode(p, v.stream, v.smem, &err);
     if (err != 0) return kd_internal_fail(ctx, KD_ECUDA, cudaGetErrorString((cudaError_t)err));
