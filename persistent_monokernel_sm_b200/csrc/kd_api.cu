@@ -73,9 +73,9 @@ Layout make_layout(const Dims& d) {
     y.vcache = take(kv);
     y.kv_bytes = 2 * kv;
     y.x = take(D * 4);
-    y.q = take((size_t)d.qd * 4);
+    y.qkv = take((size_t)d.qkv_rows * 4);  // raw q/k/v projections (repacked row order)
     y.o = take((size_t)d.qd * 4);
-    y.hdn = take((size_t)d.F * 4);
+    y.gu = take((size_t)2 * d.F * 4);  // raw gate/up projections, interleaved
     y.part = take((size_t)kMaxGrid * d.r * (d.hd + 2) * 4);
     y.ctl = take((size_t)kCtlWords * 8);
     y.tokens_in = take((size_t)d.S * 4);
@@ -93,12 +93,12 @@ struct kd_ctx {
     uint8_t* arena;
     cudaStream_t stream;
     int device;
-    int nb, smem, ns, pieces, pos_per_stage, xs_floats;
+    int nb, smem, ns, pieces, pos_per_stage, xs_floats, xown_floats;
     bool has_weights, failed;
     int pos, n_pending;
     long long launches;
     long long timeout_ns;
-    int prefetch;
+    int prefetch, inflight;
     unsigned long long* trace;
     int trace_every, trace_rows;
     char err[512];
@@ -171,8 +171,10 @@ int kd_internal_view(kd_ctx* c, kd_ctx_view* v) {
     v->stream = c->stream;
     v->device = c->device, v->nb = c->nb, v->smem = c->smem, v->ns = c->ns;
     v->pieces = c->pieces, v->pos_per_stage = c->pos_per_stage, v->xs_floats = c->xs_floats;
+    v->xown_floats = c->xown_floats;
     v->timeout_ns = c->timeout_ns;
     v->prefetch = c->prefetch;
+    v->inflight = c->inflight;
     v->has_weights = c->has_weights;
     return KD_OK;
 }
@@ -215,8 +217,10 @@ int kd_create(const kd_config* cfg, void* d_arena, size_t arena_bytes, void* str
     c->stream = (cudaStream_t)stream;
     c->timeout_ns = 1000000000LL;
     if (const char* t = getenv("KD_TIMEOUT_MS")) c->timeout_ns = atoll(t) * 1000000LL;
-    c->prefetch = 6;
+    c->prefetch = 0;
     if (const char* t = getenv("KD_PREFETCH")) c->prefetch = atoi(t);
+    c->inflight = 2;
+    if (const char* t = getenv("KD_INFLIGHT")) c->inflight = atoi(t);
     int rc = KD_OK;
     if (arena_bytes < c->lay.total || ((uintptr_t)d_arena & 255)) {
         rc = fail(c, KD_ENOMEM, "arena of %zu bytes at %p; need %zu bytes, 256-byte aligned", arena_bytes,
@@ -234,8 +238,8 @@ int kd_create(const kd_config* cfg, void* d_arena, size_t arena_bytes, void* str
         c->nb = prop.multiProcessorCount;
         if (c->nb > kMaxGrid) c->nb = kMaxGrid;
         c->pieces = c->nb / d.Hkv;
-        // attention stages: 8 positions per consumer warp (16 for hd 64), K then V rows
-        c->pos_per_stage = (d.hd == 128 ? 8 : 16) * kConsumerWarps;
+        // attention stages: 8 positions per warp of a group (16 for hd 64), K then V rows
+        c->pos_per_stage = (d.hd == 128 ? 8 : 16) * kGroupWarps;
         int xs = d.d;
         if (d.qd > xs) xs = d.qd;
         if (d.F > xs) xs = d.F;
@@ -243,12 +247,15 @@ int kd_create(const kd_config* cfg, void* d_arena, size_t arena_bytes, void* str
         if (merge > xs) xs = merge;
         if (kMaxGroup * c->pieces + kMaxGroup > xs) xs = kMaxGroup * c->pieces + kMaxGroup;  // combine weights
         c->xs_floats = (xs + 31) & ~31;
+        c->xown_floats = (d.d + c->nb - 1) / c->nb + 1;
         Params p{};
         p.xs_floats = c->xs_floats;
+        p.xown_floats = c->xown_floats;
         p.ns = 1;
         const int fixed = monokernel_smem_bytes(p) - kStageBytes;
         c->ns = (kSmemLimit - fixed) / kStageBytes;
         if (c->ns > kMaxStages) c->ns = kMaxStages;
+        c->ns -= c->ns % kGroups;  // consumer group g owns the slots g mod kGroups
         if (c->ns < 2) rc = fail(c, KD_EINVAL, "activation buffers leave no room for a pipeline");
         if (rc == KD_OK) {
             p.ns = c->ns;
@@ -375,8 +382,10 @@ int kd_decode(kd_ctx* c, int32_t n_gen, int32_t* d_tokens_out, float* d_logits_o
     p.rows_d = rows_per_stage(c->dm.F, false);
     p.rows_lm = rows_per_stage(c->dm.d, false);
     p.xs_floats = c->xs_floats;
+    p.xown_floats = c->xown_floats;
     p.timeout_ns = c->timeout_ns;
     p.prefetch = c->prefetch;
+    p.inflight = c->inflight;
     p.trace = c->trace;
     p.trace_every = c->trace_every;
     p.trace_rows = c->trace_rows;

@@ -139,6 +139,9 @@ struct Tracer {
     }
 };
 
+// Lane that performs a warp's shared-memory bookkeeping (see run_gemv).
+constexpr int kSyncLane = 31;
+
 // ------------------------------------------------------------------ schedule geometry
 // Both the producer and the consumers enumerate the same stage sequence from these.
 
@@ -221,14 +224,16 @@ struct Smem {
     uint64_t* empty;
     float* sp;              // per-stage partial sums [slot][row][warp]
     int* scnt;              // per-stage arrival counts [slot]
+    float* xown;            // the residual rows this CTA owns (updated by O and D)
+    __nv_bfloat16* kvcur;   // the current position's K and V row of the head being attended
 };
 
 // Byte offsets of the shared-memory regions; each starts on a 128-byte boundary (vector
 // loads and bulk-copy destinations need 16). Used by the kernel and for the launch size.
 struct SmemLayout {
-    size_t ring, xs, qs, rope, red, best, flag, full, empty, sp, scnt, total;
+    size_t ring, xs, qs, rope, red, best, flag, full, empty, sp, scnt, xown, kvcur, total;
 };
-__host__ __device__ inline SmemLayout smem_layout(int ns, int xs_floats) {
+__host__ __device__ inline SmemLayout smem_layout(int ns, int xs_floats, int xown_floats) {
     SmemLayout L;
     size_t off = 0;
     auto take = [&](size_t bytes) {
@@ -245,14 +250,16 @@ __host__ __device__ inline SmemLayout smem_layout(int ns, int xs_floats) {
     L.flag = take(16 * 4);
     L.full = take((size_t)kMaxStages * 8);
     L.empty = take((size_t)kMaxStages * 8);
-    L.sp = take((size_t)kMaxStages * kMaxRows * 8 * 4);
+    L.sp = take((size_t)kMaxStages * kMaxRows * 4);
     L.scnt = take((size_t)kMaxStages * 4);
+    L.xown = take((size_t)xown_floats * 4);
+    L.kvcur = take(2 * 128 * 2);
     L.total = off;
     return L;
 }
 
 __device__ __forceinline__ Smem carve(const Params& P, uint8_t* base) {
-    const SmemLayout L = smem_layout(P.ns, P.xs_floats);
+    const SmemLayout L = smem_layout(P.ns, P.xs_floats, P.xown_floats);
     Smem s;
     s.ring = base + L.ring;
     s.xs = reinterpret_cast<float*>(base + L.xs);
@@ -265,10 +272,12 @@ __device__ __forceinline__ Smem carve(const Params& P, uint8_t* base) {
     s.empty = reinterpret_cast<uint64_t*>(base + L.empty);
     s.sp = reinterpret_cast<float*>(base + L.sp);
     s.scnt = reinterpret_cast<int*>(base + L.scnt);
+    s.xown = reinterpret_cast<float*>(base + L.xown);
+    s.kvcur = reinterpret_cast<__nv_bfloat16*>(base + L.kvcur);
     return s;
 }
 
-int monokernel_smem_bytes(const Params& p) { return (int)smem_layout(p.ns, p.xs_floats).total; }
+int monokernel_smem_bytes(const Params& p) { return (int)smem_layout(p.ns, p.xs_floats, p.xown_floats).total; }
 
 // Split layout of an activation vector of length K (K % 8 == 0): element k lives at
 // ((k & 7) >> 2) * (K / 2) + (k >> 3) * 4 + (k & 3), so lane-strided 8-element chunks
@@ -381,6 +390,7 @@ __device__ void load_rmsnorm(const Smem& sm, const float* src_f32, const __nv_bf
                              const __nv_bfloat16* gain, int K, float eps) {
     const int tid = threadIdx.x;
     float ss = 0.f;
+#pragma unroll 4
     for (int k = tid * 4; k < K; k += kConsumerThreads * 4) {
         float4 v;
         if (src_f32) {
@@ -413,7 +423,24 @@ __device__ void load_rmsnorm(const Smem& sm, const float* src_f32, const __nv_bf
     consumer_sync();
 }
 
+// xs <- silu(gate) * up for the F interleaved (gate, up) pairs of the raw projection.
+__device__ void load_swiglu(const Smem& sm, const float* gu, int F) {
+#pragma unroll 4
+    for (int k = threadIdx.x * 4; k < F; k += kConsumerThreads * 4) {
+        const float4 p = __ldcg(reinterpret_cast<const float4*>(gu + 2 * k));
+        const float4 q = __ldcg(reinterpret_cast<const float4*>(gu + 2 * k + 4));
+        float4 h;
+        h.x = p.x / (1.0f + expf(-p.x)) * p.y;
+        h.y = p.z / (1.0f + expf(-p.z)) * p.w;
+        h.z = q.x / (1.0f + expf(-q.x)) * q.y;
+        h.w = q.z / (1.0f + expf(-q.z)) * q.w;
+        *reinterpret_cast<float4*>(&sm.xs[xs_index(k, F)]) = h;
+    }
+    consumer_sync();
+}
+
 __device__ void load_vector(const Smem& sm, const float* src, int K) {
+#pragma unroll 4
     for (int k = threadIdx.x * 4; k < K; k += kConsumerThreads * 4)
         *reinterpret_cast<float4*>(&sm.xs[xs_index(k, K)]) = __ldcg(reinterpret_cast<const float4*>(src + k));
     consumer_sync();
@@ -435,230 +462,177 @@ struct StepCtx {
     unsigned long long lm_best;  // running argmax key of this warp (lane 0)
 };
 
-// Sum N values per lane across the 32 lanes with log-depth exchanges that halve the
-// number of live values at each step: afterwards lane (i << (5 - log2 N)) holds the total
-// of value i (N = 1, 2, 4 or 8; 5, 5, 6 or 9 shuffles). Compile-time recursion keeps every
-// index static, so the values stay in registers.
-template <int N, int BIT>
-__device__ __forceinline__ float multi_reduce_step(const float (&v)[N], int lane) {
-    if constexpr (N == 1) {
-        float x = v[0];
-#pragma unroll
-        for (int o = BIT; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
-        return x;
-    } else {
-        constexpr int H = N / 2;
-        const bool upper = (lane & BIT) != 0;
-        float w[H];
-#pragma unroll
-        for (int i = 0; i < H; ++i) {
-            // keep the half selected by this lane's bit, send the other half to the partner
-            const float send = upper ? v[i] : v[i + H];
-            const float keep = upper ? v[i + H] : v[i];
-            w[i] = keep + __shfl_xor_sync(0xffffffffu, send, BIT);
-        }
-        return multi_reduce_step<H, BIT / 2>(w, lane);
-    }
-}
-template <int N>
-__device__ __forceinline__ float multi_reduce(const float (&v)[N]) {
-    return multi_reduce_step<N, 16>(v, threadIdx.x & 31);
-}
-
-// One warp's share of a GEMV stage: all n (<= RMAX) rows of the stage over the 8-element
-// chunks [c0, c1) of the reduction dimension, lane-strided. Each activation chunk is read
-// once and used for every row (RMAX independent accumulators). Leaves this lane's partial
-// sum of each row in v[] (reduce across lanes with multi_reduce).
-template <int RMAX>
-__device__ __forceinline__ void gemv_part(const uint8_t* st, size_t rowb, int n, int c0, int c1, const float* xs,
-                                          int K, float (&v)[RMAX]) {
-    const int lane = threadIdx.x & 31;
-    constexpr int SUB = RMAX >= 4 ? 1 : 4 / RMAX;  // accumulators per row (latency hiding)
-    float acc[RMAX][SUB];
-#pragma unroll
-    for (int r = 0; r < RMAX; ++r)
-#pragma unroll
-        for (int u = 0; u < SUB; ++u) acc[r][u] = 0.f;
-    const float4* xlo = reinterpret_cast<const float4*>(xs);
-    const float4* xhi = reinterpret_cast<const float4*>(xs + (K >> 1));
-#pragma unroll 2
-    for (int c = c0 + lane; c < c1; c += 32) {
-        const float4 x = xlo[c], y = xhi[c];
-#pragma unroll
-        for (int r = 0; r < RMAX; ++r) {
-            if (r < n) {
-                const uint4 w = *reinterpret_cast<const uint4*>(st + r * rowb + (size_t)c * 16);
-                const float f[8] = {bf_lo(w.x), bf_hi(w.x), bf_lo(w.y), bf_hi(w.y),
-                                    bf_lo(w.z), bf_hi(w.z), bf_lo(w.w), bf_hi(w.w)};
-                const float g[8] = {x.x, x.y, x.z, x.w, y.x, y.y, y.z, y.w};
-#pragma unroll
-                for (int e = 0; e < 8; ++e) acc[r][e % SUB] = fmaf(f[e], g[e], acc[r][e % SUB]);
-            }
-        }
-    }
-#pragma unroll
-    for (int r = 0; r < RMAX; ++r) {
-        float t = acc[r][0];
-#pragma unroll
-        for (int u = 1; u < SUB; ++u) t += acc[r][u];
-        v[r] = t;
-    }
-}
-
-// Phase epilogue for the rows [r0, r0 + n) of one stage; lane i holds row r0 + i's total.
-__device__ __forceinline__ void gemv_epilogue(const Params& P, const Smem& sm, int phase, int l, int r0, int n,
-                                              float tot, StepCtx& sc, float* xg) {
-    const Dims& dm = P.dm;
-    const int lane = threadIdx.x & 31;
-    if (phase == kQKV || phase == kGU) {
-        const float nb = __shfl_down_sync(0xffffffffu, tot, 1);
-        if (!(lane & 1) && lane < n) {
-            const float a = tot, b = nb;
-            const int row = r0 + lane;  // even row of a (RoPE pair | gate, up) pair
-            if (phase == kGU) {
-                float* hdn = reinterpret_cast<float*>(const_cast<uint8_t*>(P.arena) + P.lay.hdn);
-                __stcg(hdn + (row >> 1), a / (1.0f + expf(-a)) * b);
-            } else if (row < dm.qd + dm.kvd) {
-                const int hd = dm.hd;
-                const bool isq = row < dm.qd;
-                const int rr = isq ? row : row - dm.qd;
-                const int h = rr / hd, i = (rr % hd) >> 1;
-                const float2 cs = sm.rope[i];
-                const float ra_ = a * cs.x - b * cs.y;
-                const float rb_ = b * cs.x + a * cs.y;
-                if (isq) {
-                    float* q = reinterpret_cast<float*>(const_cast<uint8_t*>(P.arena) + P.lay.q);
-                    __stcg(q + h * hd + i, ra_);
-                    __stcg(q + h * hd + i + hd / 2, rb_);
-                } else {
-                    __nv_bfloat16* kc = reinterpret_cast<__nv_bfloat16*>(const_cast<uint8_t*>(P.arena) + P.lay.kcache) +
-                                        (((size_t)l * dm.Hkv + h) * dm.S + sc.p) * hd;
-                    kc[i] = __float2bfloat16_rn(ra_);
-                    kc[i + hd / 2] = __float2bfloat16_rn(rb_);
-                    fence_proxy_async_global();
-                }
-            } else {
-                const int rr = row - dm.qd - dm.kvd;
-                const int h = rr / dm.hd, j2 = rr % dm.hd;
-                __nv_bfloat16* vc = reinterpret_cast<__nv_bfloat16*>(const_cast<uint8_t*>(P.arena) + P.lay.vcache) +
-                                    (((size_t)l * dm.Hkv + h) * dm.S + sc.p) * dm.hd;
-                vc[j2] = __float2bfloat16_rn(a);
-                vc[j2 + 1] = __float2bfloat16_rn(b);
-                fence_proxy_async_global();
-            }
-        }
+// Output of one finished GEMV row (global row index `row`, value y): stored raw for the
+// Q/K/V and gate/up projections (RoPE, the KV-cache append and SwiGLU are applied where the
+// values are consumed), added into the residual for O and down (the CTA owns those rows and
+// keeps them in shared memory, so no read-back from L2), and for the LM head dumped when
+// requested and folded into this thread's running argmax.
+__device__ __forceinline__ void row_out(const Params& P, const Smem& sm, int phase, int row, float y, StepCtx& sc,
+                                        int own0) {
+    uint8_t* arena = const_cast<uint8_t*>(P.arena);
+    if (phase == kQKV) {
+        __stcg(reinterpret_cast<float*>(arena + P.lay.qkv) + row, y);
+    } else if (phase == kGU) {
+        __stcg(reinterpret_cast<float*>(arena + P.lay.gu) + row, y);
     } else if (phase == kO || phase == kD) {
-        if (lane < n) __stcg(xg + r0 + lane, __ldcg(xg + r0 + lane) + tot);
-    } else {  // LM head: dump, then this warp's running argmax (lowest index on ties)
-        if (P.dump && lane < n) __stcg(P.logits_out + (size_t)sc.t * dm.V + r0 + lane, tot);
-        unsigned long long key = lane < n ? argmax_key(tot, r0 + lane) : 0ull;
+        const float v = sm.xown[row - own0] + y;
+        sm.xown[row - own0] = v;
+        __stcg(reinterpret_cast<float*>(arena + P.lay.x) + row, v);
+    } else {
+        if (P.dump) __stcg(P.logits_out + (size_t)sc.t * P.dm.V + row, y);
+        const unsigned long long key = argmax_key(y, row);
+        if (key > sc.lm_best) sc.lm_best = key;
+    }
+}
+
+// One GEMV phase. Consumer groups take the stages of their ring slots (slot mod kGroups).
+// Within a group the R (<= 8) rows of a stage are split over its 8 warps as R rows x 8/R
+// slices of the reduction dimension; a warp keeps its slice of the activation vector in
+// registers for the whole phase, so a stage costs it one 16-byte shared-memory load and 8
+// FMAs per chunk. When a warp owns a whole row (R = 8) it finishes the row itself; when rows
+// are split, the warps' partial sums meet in shared memory and the last warp of the stage
+// adds them in a fixed order. Either way the per-row epilogue (row_out) is a store or two.
+// A wait that gives up marks `ok` false and the warp skips the work of the remaining
+// stages, but it still reaches every named barrier; the next grid barrier then reports
+// the failure to the whole CTA at once.
+__device__ __noinline__ void run_gemv(const Params& P, const Smem& sm_ref, unsigned long long* ctl, int phase, int l,
+                                      Ring& rg_ref, StepCtx& sc_ref, bool& ok_ref, Tracer& tr) {
+    // A separate function (its own register allocation) working on register copies of the
+    // caller's state, written back at the end.
+    const Smem sm = sm_ref;
+    Ring rg = rg_ref;
+    StepCtx sc = sc_ref;
+    bool ok = ok_ref;
+    const Gemv g = gemv_geom(P, phase, l, blockIdx.x);
+    const int nst = gemv_stages(g);
+    const int ns = P.ns;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int group = warp / kGroupWarps, gw = warp % kGroupWarps;
+    const int KS = kGroupWarps / g.R;  // slices per row (rows_per_stage gives R in {1, 2, 4, 8})
+    const int row = gw / KS, ks = gw % KS;
+    const int nch = g.K >> 3;
+    const int c0 = nch * ks / KS, c1 = nch * (ks + 1) / KS;  // at most 32 * kMaxChunks chunks
+    const size_t rowb = (size_t)g.K * 2;
+    const int own0 = (int)((long long)P.dm.d * blockIdx.x / P.nb);
+    unsigned long long* waited = threadIdx.x == 0 ? &tr.waited : nullptr;
+
+    // this lane's activation chunks: c = c0 + lane + 32 i
+    float xr[kMaxChunks][8];
+    const float4* xlo = reinterpret_cast<const float4*>(sm.xs);
+    const float4* xhi = reinterpret_cast<const float4*>(sm.xs + (g.K >> 1));
+#pragma unroll
+    for (int i = 0; i < kMaxChunks; ++i) {
+        const int c = c0 + lane + 32 * i;
+        const float4 a = c < c1 ? xlo[c] : make_float4(0.f, 0.f, 0.f, 0.f);
+        const float4 b = c < c1 ? xhi[c] : make_float4(0.f, 0.f, 0.f, 0.f);
+        xr[i][0] = a.x, xr[i][1] = a.y, xr[i][2] = a.z, xr[i][3] = a.w;
+        xr[i][4] = b.x, xr[i][5] = b.y, xr[i][6] = b.z, xr[i][7] = b.w;
+    }
+
+    // Stages are taken two at a time (this group's next two): their 16 chunk loads and the
+    // two cross-lane reductions interleave, and the per-stage bookkeeping is paid once per pair.
+    auto dot_row = [&](const uint8_t* wrow, float& s) {
+        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll
+        for (int i = 0; i < kMaxChunks; ++i) {
+            const int c = c0 + lane + 32 * i;
+            if (c < c1) {
+                const uint4 w = *reinterpret_cast<const uint4*>(wrow + (size_t)c * 16);
+                a0 = fmaf(bf_lo(w.x), xr[i][0], a0);
+                a1 = fmaf(bf_hi(w.x), xr[i][1], a1);
+                a2 = fmaf(bf_lo(w.y), xr[i][2], a2);
+                a3 = fmaf(bf_hi(w.y), xr[i][3], a3);
+                a0 = fmaf(bf_lo(w.z), xr[i][4], a0);
+                a1 = fmaf(bf_hi(w.z), xr[i][5], a1);
+                a2 = fmaf(bf_lo(w.w), xr[i][6], a2);
+                a3 = fmaf(bf_hi(w.w), xr[i][7], a3);
+            }
+        }
+        s = (a0 + a1) + (a2 + a3);
+    };
+    // per-stage completion: release the slot and put the row(s) out
+    auto finish = [&](const Ring& at_rg, int r0, int n, float part) {
+        if (KS == 1) {  // this warp owns the whole row
+            __syncwarp();
+            if (lane == kSyncLane) mbar_arrive(smem_u32(&sm.empty[at_rg.slot]));  // done with the stage
+            if (lane == 0 && row < n) row_out(P, sm, phase, r0 + row, part, sc, own0);
+            return;
+        }
+        float* sp = sm.sp + (size_t)at_rg.slot * kMaxRows;  // [row * KS + slice]: R * KS = 8 values
+        int last = 0;
+        if (lane == kSyncLane) {
+            if (row < n) sp[row * KS + ks] = part;
+            __threadfence_block();
+            last = atomicAdd(&sm.scnt[at_rg.slot], 1) == kGroupWarps - 1;
+            if (!last) mbar_arrive(smem_u32(&sm.empty[at_rg.slot]));  // done with the stage
+        }
+        if (!__shfl_sync(0xffffffffu, last, kSyncLane)) return;
+        // last warp of the stage: row totals (lane = row) in a fixed order, release, rows out
+        __threadfence_block();
+        float tot = 0.f;
+        if (lane < n)
+            for (int q = 0; q < KS; ++q) tot += sp[lane * KS + q];
+        __syncwarp();
+        if (lane == kSyncLane) {
+            sm.scnt[at_rg.slot] = 0;
+            mbar_arrive(smem_u32(&sm.empty[at_rg.slot]));  // partial sums read: the slot may refill
+        }
+        if (lane < n) row_out(P, sm, phase, r0 + lane, tot, sc, own0);
+    };
+
+    int j = 0;
+    while (j < nst) {
+        // this group's next stage, and the one after it
+        while (j < nst && rg.slot % kGroups != group) {
+            ++j;
+            rg.advance(ns);
+        }
+        if (j >= nst) break;
+        const int ja = j;
+        const Ring ra = rg;
+        ++j;
+        rg.advance(ns);
+        while (j < nst && rg.slot % kGroups != group) {
+            ++j;
+            rg.advance(ns);
+        }
+        const bool two = j < nst;
+        const int jb = j;
+        const Ring rb = rg;
+        if (two) {
+            ++j;
+            rg.advance(ns);
+        }
+        if (!ok) continue;
+        if (!wait_full(sm, ra, P, ctl, waited) || (two && !wait_full(sm, rb, P, ctl, waited))) {
+            ok = false;
+            continue;
+        }
+        const int ra0 = g.row0 + ja * g.R, na = min(g.R, g.row1 - ra0);
+        const int rb0 = g.row0 + jb * g.R, nb = two ? min(g.R, g.row1 - rb0) : 0;
+        float pa = 0.f, pb = 0.f;
+        if (row < na) dot_row(sm.ring + (size_t)ra.slot * kStageBytes + row * rowb, pa);
+        if (row < nb) dot_row(sm.ring + (size_t)rb.slot * kStageBytes + row * rowb, pb);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            pa += __shfl_xor_sync(0xffffffffu, pa, o);
+            pb += __shfl_xor_sync(0xffffffffu, pb, o);
+        }
+        finish(ra, ra0, na, pa);
+        if (two) finish(rb, rb0, nb, pb);
+    }
+    rg_ref = rg;
+    ok_ref = ok;
+    // LM head: fold the lanes' running argmax into lane 0's (lowest index on ties)
+    if (phase == kLM) {
+        unsigned long long key = sc.lm_best;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
             const unsigned long long other = __shfl_xor_sync(0xffffffffu, key, o);
             key = other > key ? other : key;
         }
-        if (lane == 0 && key > sc.lm_best) sc.lm_best = key;
+        sc_ref.lm_best = key;
     }
-}
-
-// One GEMV phase. Every consumer warp takes part in every stage: warp w reduces all R rows
-// of the stage over the w-th seventh of the reduction dimension and writes its R partial
-// sums to shared memory; the last warp to finish the stage adds the seven slices in a fixed
-// order, releases the stage, and applies the phase's epilogue to the R rows.
-// A wait that gives up marks `ok` false and the warp skips the work of the remaining
-// stages, but it still reaches every named barrier; the next grid barrier then reports
-// the failure to the whole CTA at once.
-template <int RMAX>
-__device__ __noinline__ void run_gemv_t(const Params& P, const Smem& sm_ref, unsigned long long* ctl, int phase, int l,
-                                       const Gemv& g_ref, Ring& rg_ref, StepCtx& sc_ref, bool& ok_ref, Tracer& tr) {
-    // This is a separate function (its own register allocation); work on register copies of
-    // the caller's state and write back at the end.
-    const Smem sm = sm_ref;
-    const Gemv g = g_ref;
-    Ring rg = rg_ref;
-    StepCtx sc = sc_ref;
-    bool ok = ok_ref;
-    constexpr int SHIFT = RMAX == 8 ? 2 : RMAX == 4 ? 3 : RMAX == 2 ? 4 : 5;
-    const Dims& dm = P.dm;
-    const int nst = gemv_stages(g);
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int nch = g.K >> 3;
-    const int c0 = nch * warp / kConsumerWarps, c1 = nch * (warp + 1) / kConsumerWarps;
-    const size_t rowb = (size_t)g.K * 2;
-    float* xg = reinterpret_cast<float*>(const_cast<uint8_t*>(P.arena) + P.lay.x);
-    unsigned long long* waited = threadIdx.x == 0 ? &tr.waited : nullptr;
-    // Two stages in flight per warp: the loads and FMAs of stage j + 1 are issued before the
-    // cross-lane reduction and epilogue of stage j, hiding the latter's latency.
-    float cur[RMAX], nxt[RMAX];
-    Ring rj = rg;  // ring position of stage j
-    if (nst > 0 && ok) {
-        if (!wait_full(sm, rj, P, ctl, waited)) ok = false;
-        else gemv_part<RMAX>(sm.ring + (size_t)rj.slot * kStageBytes, rowb, min(g.R, g.row1 - g.row0), c0, c1, sm.xs,
-                             g.K, cur);
-    }
-    for (int j = 0; j < nst; ++j) {
-        Ring rn = rj;
-        rn.advance(P.ns);
-        if (!ok) {
-            rj = rn;
-            continue;
-        }
-        if (j + 1 < nst) {
-            if (!wait_full(sm, rn, P, ctl, waited)) {
-                ok = false;
-                rj = rn;
-                continue;
-            }
-            const int rn0 = g.row0 + (j + 1) * g.R;
-            gemv_part<RMAX>(sm.ring + (size_t)rn.slot * kStageBytes, rowb, min(g.R, g.row1 - rn0), c0, c1, sm.xs, g.K,
-                            nxt);
-        }
-        const int r0 = g.row0 + j * g.R;
-        const int n = min(g.R, g.row1 - r0);
-        const float part = multi_reduce<RMAX>(cur);
-        float* sp = sm.sp + (size_t)rj.slot * (kMaxRows * 8);  // [row][warp], rows padded to 8 warps
-        const int prow = lane >> SHIFT;
-        if ((lane & ((1 << SHIFT) - 1)) == 0 && prow < n) sp[prow * 8 + warp] = part;
-        __syncwarp();
-        int last = 0;
-        if (lane == 0) {
-            __threadfence_block();
-            last = atomicAdd(&sm.scnt[rj.slot], 1) == kConsumerWarps - 1;
-            if (!last) mbar_arrive(smem_u32(&sm.empty[rj.slot]));  // done with the stage
-        }
-        if (__shfl_sync(0xffffffffu, last, 0)) {
-            // ---- last warp of this stage: row totals (lane = row), release, epilogue
-            __threadfence_block();
-            float tot = 0.f;
-            if (lane < n) {
-                const float4 a = *reinterpret_cast<const float4*>(sp + lane * 8);
-                const float4 b = *reinterpret_cast<const float4*>(sp + lane * 8 + 4);
-                static_assert(kConsumerWarps == 7, "row totals add 7 warp slices");
-                tot = ((a.x + a.y) + (a.z + a.w)) + ((b.x + b.y) + b.z);
-            }
-            __syncwarp();
-            if (lane == 0) {
-                sm.scnt[rj.slot] = 0;
-                mbar_arrive(smem_u32(&sm.empty[rj.slot]));  // partial sums read: the slot may refill
-            }
-            gemv_epilogue(P, sm, phase, l, r0, n, tot, sc, xg);
-        }
-#pragma unroll
-        for (int r = 0; r < RMAX; ++r) cur[r] = nxt[r];
-        rj = rn;
-    }
-    rg_ref = rj;
-    sc_ref.lm_best = sc.lm_best;
-    ok_ref = ok;
-}
-
-__device__ void run_gemv(const Params& P, const Smem& sm, unsigned long long* ctl, int phase, int l, Ring& rg,
-                         StepCtx& sc, bool& ok, Tracer& tr) {
-    const Gemv g = gemv_geom(P, phase, l, blockIdx.x);
-    if (g.R <= 1) run_gemv_t<1>(P, sm, ctl, phase, l, g, rg, sc, ok, tr);
-    else if (g.R <= 2) run_gemv_t<2>(P, sm, ctl, phase, l, g, rg, sc, ok, tr);
-    else if (g.R <= 4) run_gemv_t<4>(P, sm, ctl, phase, l, g, rg, sc, ok, tr);
-    else run_gemv_t<8>(P, sm, ctl, phase, l, g, rg, sc, ok, tr);  // rows_per_stage caps R at 8
 }
 
 // Loads that read either the shared-memory ring or, for the current position, the cache
@@ -699,8 +673,40 @@ __device__ __noinline__ void run_attention(const Params& P, const Smem& sm_ref, 
     if (at.g < 0) return;  // uniform across the CTA
     const int r = dm.r, A = P.attn_pieces;
     const float qscale = 1.4426950408889634f / sqrtf((float)HD);  // log2(e) / sqrt(hd)
-    const float* qg = reinterpret_cast<const float*>(P.arena + P.lay.q) + (size_t)at.g * r * HD;
-    for (int i = tid; i < r * HD; i += kConsumerThreads) sm.qs[i] = __ldcg(qg + i) * qscale;
+    // The Q/K/V projections arrive raw, q and k rows in RoPE-pair order (row 2i = dim i,
+    // row 2i + 1 = dim i + hd/2). Rotate this group's q heads at position p while loading.
+    const float* raw = reinterpret_cast<const float*>(P.arena + P.lay.qkv);
+    const float* qg = raw + (size_t)at.g * r * HD;
+    for (int t = tid; t < r * HD / 2; t += kConsumerThreads) {
+        const int hh = t / (HD / 2), i = t % (HD / 2);
+        const float a = __ldcg(qg + hh * HD + 2 * i), b = __ldcg(qg + hh * HD + 2 * i + 1);
+        const float2 cs = sm.rope[i];
+        sm.qs[hh * HD + i] = (a * cs.x - b * cs.y) * qscale;
+        sm.qs[hh * HD + i + HD / 2] = (b * cs.x + a * cs.y) * qscale;
+    }
+    // The piece that holds position p appends that position's K (rotated) and V to the
+    // cache, rounded to bf16, and keeps a copy for its own pass below.
+    const bool has_current = at.b > sc.p;
+    if (has_current) {
+        const size_t off = (((size_t)l * dm.Hkv + at.g) * dm.S + sc.p) * HD;
+        __nv_bfloat16* kc = reinterpret_cast<__nv_bfloat16*>(const_cast<uint8_t*>(P.arena) + P.lay.kcache) + off;
+        __nv_bfloat16* vc = reinterpret_cast<__nv_bfloat16*>(const_cast<uint8_t*>(P.arena) + P.lay.vcache) + off;
+        const float* kr = raw + dm.qd + (size_t)at.g * HD;
+        const float* vr = raw + dm.qd + dm.kvd + (size_t)at.g * HD;
+        for (int i = tid; i < HD / 2; i += kConsumerThreads) {
+            const float a = __ldcg(kr + 2 * i), b = __ldcg(kr + 2 * i + 1);
+            const float2 cs = sm.rope[i];
+            const __nv_bfloat16 k0 = __float2bfloat16_rn(a * cs.x - b * cs.y);
+            const __nv_bfloat16 k1 = __float2bfloat16_rn(b * cs.x + a * cs.y);
+            kc[i] = k0, kc[i + HD / 2] = k1;
+            sm.kvcur[i] = k0, sm.kvcur[i + HD / 2] = k1;
+            const __nv_bfloat16 v0 = __float2bfloat16_rn(__ldcg(vr + 2 * i));
+            const __nv_bfloat16 v1 = __float2bfloat16_rn(__ldcg(vr + 2 * i + 1));
+            vc[2 * i] = v0, vc[2 * i + 1] = v1;
+            sm.kvcur[HD + 2 * i] = v0, sm.kvcur[HD + 2 * i + 1] = v1;
+        }
+        fence_proxy_async_global();  // later bulk copies (async proxy) read these rows
+    }
     consumer_sync();
     if (tid == 0) tr.mark(4);
 
@@ -796,64 +802,31 @@ __device__ __noinline__ void run_attention(const Params& P, const Smem& sm_ref, 
         }
     };
 
-    // This warp's positions of each stage: [n * w / W, n * (w + 1) / W) of the stage's n.
-    // With hd 128 that is at most 8, and two consecutive stages share one pass; with hd 64
-    // it is at most 16, split over one pass.
+    // Stages alternate between the two groups (ring-slot parity); within a stage, warp gw of
+    // the group takes positions [n * gw / 8, n * (gw + 1) / 8): at most 8 with hd 128, at
+    // most 16 (two blocks of one pass) with hd 64.
     const int nst = attn_stages(P, at);
+    const int group = warp / kGroupWarps, gw = warp % kGroupWarps;
     unsigned long long* waited = tid == 0 ? &tr.waited : nullptr;
-    for (int j = 0; j < nst && ok;) {
+    for (int j = 0; j < nst; ++j, rg.advance(P.ns)) {
+        if (rg.slot % kGroups != group || !ok) continue;  // group g: slots g mod kGroups
         if (!wait_full(sm, rg, P, ctl, waited)) {
             ok = false;
-            break;
+            continue;
         }
         const int s0 = at.a + j * P.pos_per_stage;
         const int n = min(P.pos_per_stage, at.tma_end - s0);
         const __nv_bfloat16* st = reinterpret_cast<const __nv_bfloat16*>(sm.ring + (size_t)rg.slot * kStageBytes);
-        const int p0 = n * warp / kConsumerWarps, p1 = n * (warp + 1) / kConsumerWarps;
+        const int p0 = n * gw / kGroupWarps, p1 = n * (gw + 1) / kGroupWarps;
         const __nv_bfloat16* ka = st + (size_t)p0 * HD;
         const __nv_bfloat16* va = st + (size_t)(n + p0) * HD;
-        const int na = min(8, p1 - p0);
-        Ring r2 = rg;
-        r2.advance(P.ns);
-        if (p1 - p0 > 8) {  // hd 64: both blocks from this stage
-            pass2(ka, va, na, ka + (size_t)8 * HD, va + (size_t)8 * HD, p1 - p0 - 8, false);
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&sm.empty[rg.slot]));
-            rg = r2;
-            j += 1;
-        } else if (j + 1 < nst) {  // pair with the next stage
-            if (!wait_full(sm, r2, P, ctl, waited)) {
-                ok = false;
-                break;
-            }
-            const int s1 = at.a + (j + 1) * P.pos_per_stage;
-            const int n1 = min(P.pos_per_stage, at.tma_end - s1);
-            const __nv_bfloat16* st1 = reinterpret_cast<const __nv_bfloat16*>(sm.ring + (size_t)r2.slot * kStageBytes);
-            const int q0 = n1 * warp / kConsumerWarps, q1 = n1 * (warp + 1) / kConsumerWarps;
-            if (na > 0) pass2(ka, va, na, st1 + (size_t)q0 * HD, st1 + (size_t)(n1 + q0) * HD, q1 - q0, false);
-            __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(smem_u32(&sm.empty[rg.slot]));
-                mbar_arrive(smem_u32(&sm.empty[r2.slot]));
-            }
-            r2.advance(P.ns);
-            rg = r2;
-            j += 2;
-        } else {
-            if (na > 0) pass2(ka, va, na, ka, va, 0, false);
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&sm.empty[rg.slot]));
-            rg = r2;
-            j += 1;
-        }
+        const int na = min(8, p1 - p0), nb = p1 - p0 - na;
+        if (na > 0) pass2(ka, va, na, ka + (size_t)8 * HD, va + (size_t)8 * HD, nb, false);
+        __syncwarp();
+        if (lane == kSyncLane) mbar_arrive(smem_u32(&sm.empty[rg.slot]));
     }
-    // the current position, written by this step's QKV phase, read straight from the cache
-    if (at.b > sc.p && warp == kConsumerWarps - 1) {
-        const size_t off = (((size_t)l * dm.Hkv + at.g) * dm.S + sc.p) * HD;
-        const __nv_bfloat16* kp = reinterpret_cast<const __nv_bfloat16*>(P.arena + P.lay.kcache) + off;
-        const __nv_bfloat16* vp = reinterpret_cast<const __nv_bfloat16*>(P.arena + P.lay.vcache) + off;
-        pass2(kp, vp, 1, kp, vp, 0, true);
-    }
+    // the current position, appended above
+    if (has_current && warp == kConsumerWarps - 1) pass2(sm.kvcur, sm.kvcur + HD, 1, sm.kvcur, sm.kvcur + HD, 0, false);
 
     // merge the warps' states (xs is free during attention)
     if (tid == 0) tr.mark(5);
@@ -1059,6 +1032,25 @@ struct Producer {
         }
     }
 
+    // Keep at most P.inflight issued stages in flight: wait until stage k - inflight has
+    // landed. (Its slot cannot have been refilled yet, so its full-barrier phase is unambiguous.)
+    __device__ bool wait_landed() {
+        const int kk = k - P.inflight;
+        if (P.inflight <= 0 || kk < 0 || P.inflight >= P.ns) return true;
+        const uint32_t a = smem_u32(&sm.full[kk % P.ns]);
+        const uint32_t par = (uint32_t)((kk / P.ns) & 1);
+        if (mbar_try_wait(a, par)) return true;
+        const uint64_t t0 = globaltimer();
+        for (;;) {
+            if (mbar_wait_hint(a, par)) return true;
+            if (read_status(ctl) != 0) return false;
+            if (globaltimer() - t0 > (uint64_t)P.timeout_ns) {
+                raise_timeout(ctl, where_code(kWhereEmpty, 0x80 | (kk % P.ns)));
+                return false;
+            }
+        }
+    }
+
     // Wait until at least `need` grid barriers of this launch have completed.
     __device__ bool wait_epochs(long long need) {
         if (seen_epochs >= need) return true;
@@ -1085,10 +1077,12 @@ struct Producer {
         uint32_t b1, b2;
         int kv_last;
         cur.stage(P, s1, b1, s2, b2, kv_last);
-        if (kv_last >= P.pos0) {  // written earlier in this launch: wait for its QKV barrier
-            const long long need = barriers_before_step(P, kv_last - P.pos0) + 5ll * cur.l + 1;
+        if (kv_last >= P.pos0) {  // written earlier in this launch: wait for the barrier after
+            // the attention phase (which appends the row) of the step that wrote it
+            const long long need = barriers_before_step(P, kv_last - P.pos0) + 5ll * cur.l + 2;
             if (!wait_epochs(need)) return false;
         }
+        if (!wait_landed()) return false;
         if (!wait_empty()) return false;
         const uint32_t fb = smem_u32(&sm.full[slot]);
         const uint32_t dst = smem_u32(sm.ring + (size_t)slot * kStageBytes);
@@ -1160,7 +1154,7 @@ __global__ void __launch_bounds__(kThreads, 1) monokernel(const __grid_constant_
     if (tid == 0) {
         for (int s = 0; s < P.ns; ++s) {
             mbar_init(smem_u32(&sm.full[s]), 1);
-            mbar_init(smem_u32(&sm.empty[s]), kConsumerWarps);  // every consumer warp releases
+            mbar_init(smem_u32(&sm.empty[s]), kGroupWarps);  // every warp of the slot's group releases
             sm.scnt[s] = 0;
         }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -1225,7 +1219,11 @@ __global__ void __launch_bounds__(kThreads, 1) monokernel(const __grid_constant_
         consumer_sync();
         const int tok = sm.flag[2];
         const __nv_bfloat16* erow = embed + (size_t)tok * dm.d;
-        for (int i = own0 + tid; i < own1; i += kConsumerThreads) __stcg(xg + i, __bfloat162float(erow[i]));
+        for (int i = own0 + tid; i < own1; i += kConsumerThreads) {
+            const float v = __bfloat162float(erow[i]);
+            sm.xown[i - own0] = v;  // the residual rows this CTA updates in O and D
+            __stcg(xg + i, v);
+        }
 
         for (int l = 0; l < dm.L && ok; ++l) {
             sc.l = l;
@@ -1258,7 +1256,7 @@ __global__ void __launch_bounds__(kThreads, 1) monokernel(const __grid_constant_
             if (tid == 0) tr.mark(1);
             run_gemv(P, sm, ctl, kGU, l, rg, sc, ok, tr);
             if (!(ok = grid_sync(sm, epoch, base, P, ctl, ok, tr))) break;
-            load_vector(sm, reinterpret_cast<const float*>(P.arena + P.lay.hdn), dm.F);
+            load_swiglu(sm, reinterpret_cast<const float*>(P.arena + P.lay.gu), dm.F);
             if (tid == 0) tr.mark(1);
             run_gemv(P, sm, ctl, kD, l, rg, sc, ok, tr);
             if (!(ok = grid_sync(sm, epoch, base, P, ctl, ok, tr))) break;

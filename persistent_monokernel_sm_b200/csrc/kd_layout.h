@@ -10,10 +10,13 @@ namespace kd {
 // Pipeline: one producer warp streams weight / KV tiles into a ring of shared-memory
 // stages with 1-D bulk copies; consumer warps each take whole stages round-robin.
 constexpr int kStageBytes = 32768;
-constexpr int kConsumerWarps = 7;  // + 1 producer warp = 256 threads: the full register file
+constexpr int kGroupWarps = 8;                      // warps that share one pipeline stage
+constexpr int kGroups = 1;                          // groups take alternate stages (slot parity)
+constexpr int kConsumerWarps = kGroupWarps * kGroups;  // + 1 producer warp
 constexpr int kConsumerThreads = 32 * kConsumerWarps;
 constexpr int kThreads = kConsumerThreads + 32;
-constexpr int kMaxRows = 8;       // rows of one GEMV stage (register accumulators)
+constexpr int kMaxRows = 8;       // rows of one GEMV stage (one per warp of a group)
+constexpr int kMaxChunks = 8;     // 16-byte weight chunks per lane per row slice (x kept in registers)
 constexpr int kMaxGroup = 8;      // q heads per kv head
 constexpr int kMaxKvHeads = 16;
 constexpr int kMaxStages = 8;
@@ -42,18 +45,22 @@ struct Layout {
     size_t layer0, layer_stride;
     size_t l_attn_norm, l_ffn_norm, l_wqkv, l_wo, l_wgu, l_wd;  // within a layer block
     size_t kcache, vcache;                                        // [L][Hkv][S][hd] bf16
-    size_t x, q, o, hdn, part;                                    // fp32 scratch
+    size_t x, qkv, o, gu, part;                                   // fp32 scratch
     size_t ctl, tokens_in, tokens_out;
     size_t weights_end, kv_bytes, total;
 };
 
-// Rows per pipeline stage of one GEMV phase with reduction length K (bf16 elements);
-// `paired` phases keep row pairs (RoPE pairs, gate/up pairs) inside one stage.
+// Rows per pipeline stage of one GEMV phase with reduction length K (bf16 elements): the
+// largest power of two <= 8 whose rows fit a stage. A group of 8 warps then splits the
+// stage exactly as R rows x 8/R slices, each slice at most 2048 elements (8 chunks per
+// lane). Paired phases (RoPE pairs, gate/up pairs) always get R >= 2 since K <= 8192.
 inline int rows_per_stage(int K, bool paired) {
     int r = kStageBytes / (2 * K);
     if (r > kMaxRows) r = kMaxRows;
-    if (paired) r &= ~1;
-    return r;
+    int p2 = 1;
+    while (p2 * 2 <= r) p2 *= 2;
+    (void)paired;
+    return p2;
 }
 
 struct Params {
@@ -76,8 +83,10 @@ struct Params {
     int pos_per_stage;
     int rows_qkv, rows_o, rows_gu, rows_d, rows_lm;  // rows per stage of each GEMV phase
     int xs_floats;                                    // activation buffer (floats)
+    int xown_floats;                                  // this CTA's residual rows (floats)
     long long timeout_ns;
     int prefetch;  // stages the producer pulls into L2 ahead of the shared-memory ring
+    int inflight;  // at most this many issued stages not yet landed (bounds memory queueing)
     // optional trace: CTAs with blockIdx.x % trace_every == 0 record per-phase timestamps
     unsigned long long* trace;
     int trace_every, trace_rows;  // rows per traced CTA (4 words each)
@@ -98,9 +107,9 @@ struct kd_ctx_view {
     const Layout* lay;
     uint8_t* arena;
     void* stream;
-    int device, nb, smem, ns, pieces, pos_per_stage, xs_floats;
+    int device, nb, smem, ns, pieces, pos_per_stage, xs_floats, xown_floats;
     long long timeout_ns;
-    int prefetch;
+    int prefetch, inflight;
     bool has_weights;
 };
 int monokernel_smem_bytes(const Params& p);

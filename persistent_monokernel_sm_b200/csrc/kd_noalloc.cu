@@ -70,8 +70,8 @@ extern "C" int kd_decode_noalloc(kd_ctx* ctx, const int32_t* d_tokens, int32_t n
         off = up256(off + bytes);
         return at;
     };
-    const size_t o_x = take((size_t)dm.d * 4), o_q = take((size_t)dm.qd * 4), o_o = take((size_t)dm.qd * 4);
-    const size_t o_hdn = take((size_t)dm.F * 4);
+    const size_t o_x = take((size_t)dm.d * 4), o_q = take((size_t)dm.qkv_rows * 4), o_o = take((size_t)dm.qd * 4);
+    const size_t o_hdn = take((size_t)2 * dm.F * 4);
     const size_t o_part = take((size_t)v.nb * dm.r * (dm.hd + 2) * 4);
     const size_t o_ctl = take((size_t)kCtlWords * 8);
     const size_t o_tok = take((size_t)n_tokens * 4);
@@ -106,7 +106,7 @@ extern "C" int kd_decode_noalloc(kd_ctx* ctx, const int32_t* d_tokens, int32_t n
     Params p{};
     p.arena = v.arena;
     p.lay = *v.lay;
-    p.lay.x = rel(o_x), p.lay.q = rel(o_q), p.lay.o = rel(o_o), p.lay.hdn = rel(o_hdn);
+    p.lay.x = rel(o_x), p.lay.qkv = rel(o_q), p.lay.o = rel(o_o), p.lay.gu = rel(o_hdn);
     p.lay.part = rel(o_part), p.lay.ctl = rel(o_ctl), p.lay.tokens_in = rel(o_tok);
     p.dm = dm;
     p.steps = steps;
@@ -126,8 +126,10 @@ extern "C" int kd_decode_noalloc(kd_ctx* ctx, const int32_t* d_tokens, int32_t n
     p.rows_d = rows_per_stage(dm.F, false);
     p.rows_lm = rows_per_stage(dm.d, false);
     p.xs_floats = v.xs_floats;
+    p.xown_floats = v.xown_floats;
     p.timeout_ns = v.timeout_ns;
     p.prefetch = v.prefetch;
+    p.inflight = v.inflight;
     int err = 0;
     launch_decode(p, v.stream, v.smem, &err);
     if (err != 0) return kd_internal_fail(ctx, KD_ECUDA, cudaGetErrorString((cudaError_t)err));
