@@ -33,8 +33,9 @@
  *
  * Errors. Functions return KD_OK (0) or a negative KD_E* code. Argument, capacity and
  * co-residency errors are detected on the host before anything is launched. Errors the
- * kernel detects (a wait that exceeded its time limit) are reported by kd_sync; after one,
- * the handle refuses kd_decode until kd_reset. kd_last_error() describes the last error.
+ * kernel detects (a wait that exceeded its time limit, a token id outside the vocabulary)
+ * are reported by kd_sync; after one, the handle refuses kd_decode until kd_reset.
+ * kd_last_error() describes the last error.
  */
 #ifndef KD_H
 #define KD_H
@@ -54,7 +55,9 @@ enum {
     KD_ECOOP = -4,     /* the kernel cannot have one CTA resident on every SM */
     KD_ECUDA = -5,     /* a CUDA runtime call failed (message in kd_last_error) */
     KD_ETIMEOUT = -6,  /* a device-side wait exceeded its limit; the kernel unwound */
-    KD_ESTATE = -7     /* call out of order: no weights, nothing pending, or failed run */
+    KD_ESTATE = -7,    /* call out of order: no weights, nothing pending, or failed run */
+    KD_ETOKEN = -8     /* a token id outside [0, vocab) reached the kernel, which stopped
+                          before reading any embedding row for it */
 };
 
 /* Model shape. Limits: n_layers >= 1; head_dim in {64, 128}; n_heads a multiple of
@@ -139,7 +142,7 @@ int kd_generate(kd_ctx *ctx, const int32_t *h_tokens, int32_t n_tokens, int32_t 
                 int32_t n_gen, int32_t *h_tokens_out);
 
 /* Wait for the stream, then return the device status of the last decode (KD_OK,
- * KD_ETIMEOUT) or a CUDA error. */
+ * KD_ETIMEOUT, KD_ETOKEN) or a CUDA error. */
 int kd_sync(kd_ctx *ctx);
 
 /* kd_decode without device working memory of its own: the pages have no counterpart; this

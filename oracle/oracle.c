@@ -6,8 +6,8 @@
  * benchmark's CPU-baseline leg load this library. The CUDA decode library never links,
  * calls or reads it, and the two share no source, header, table or constant generator.
  *
- * What it computes. The pages describe the decode path as one program that covers
- * "MatMul, attention, normalization and sampling" for one request, one token at a time
+ * What it computes. The pages describe the decode path as one program that covers the
+ * matrix products, attention, normalisation and sampling for one request, one token at a time
  * ("Breaking the memory wall: 3,000 tokens/s on standard GPUs", agentlenshq.com, section
  * "1. The Monokernel Runtime"; "3000 tokens per second: how to speed up LLMs on ordinary
  * GPUs", aikraft.ru, section 04 "Monokernel and optimized GPU code"), and they say the

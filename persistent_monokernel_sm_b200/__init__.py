@@ -20,7 +20,8 @@ __all__ = ["KdError", "kd_config", "kd_weights", "kd_info", "load_library", "Dec
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkd.so")
 
 ERRORS = {0: "KD_OK", -1: "KD_EINVAL", -2: "KD_ENOMEM", -3: "KD_ECAPACITY", -4: "KD_ECOOP",
-          -5: "KD_ECUDA", -6: "KD_ETIMEOUT", -7: "KD_ESTATE"}
+          -5: "KD_ECUDA", -6: "KD_ETIMEOUT", -7: "KD_ESTATE",
+          -8: "KD_ETOKEN"}
 
 
 class kd_config(ctypes.Structure):

@@ -1,6 +1,8 @@
 // kd_api.cu -- host side of libkd: configuration checks, the arena layout, weight repacking
 // into the streaming layout, and the C ABI declared in include/kd.h.
 #include <cuda_runtime.h>
+#include <vector>
+#include <math.h>
 #include <stdarg.h>
 #include <stdio.h>
 #include <stdlib.h>
@@ -68,6 +70,7 @@ Layout make_layout(const Dims& d) {
     y.layer_stride = lo;
     off = y.layer0 + (size_t)d.L * y.layer_stride;
     y.weights_end = off;
+    y.rope = take((size_t)d.S * (d.hd / 2) * 8);  // RoPE table, filled by kd_load_weights
     const size_t kv = (size_t)d.L * d.Hkv * d.S * d.hd * 2;
     y.kcache = take(kv);
     y.vcache = take(kv);
@@ -261,7 +264,7 @@ int kd_create(const kd_config* cfg, void* d_arena, size_t arena_bytes, void* str
             p.ns = c->ns;
             c->smem = monokernel_smem_bytes(p);
             int per_sm = 0;
-            int e = monokernel_occupancy(c->smem, &per_sm);
+            int e = monokernel_occupancy(d.hd, d.r, c->smem, &per_sm);
             if (e != 0) rc = fail(c, KD_ECUDA, "occupancy query failed: %s", cudaGetErrorString((cudaError_t)e));
             else if (per_sm < 1)
                 rc = fail(c, KD_ECOOP, "monokernel cannot be resident (smem %d bytes)", c->smem);
@@ -308,6 +311,23 @@ int kd_load_weights(kd_ctx* c, const kd_weights* w) {
                                                   (const uint16_t*)w->wu, d);
     KD_CUDA(c, cudaGetLastError());
     c->launches += 2;
+    // RoPE table: (cos, sin) of position p times frequency theta^(-2i/hd), formed in double
+    // and rounded to float, for every position the cache can hold; the kernel reads one row
+    // per step.
+    {
+        const int half = d.hd / 2;
+        std::vector<float> tab((size_t)d.S * half * 2);
+        for (int i = 0; i < half; ++i) {
+            const double freq = pow((double)d.theta, -2.0 * (double)i / (double)d.hd);
+            for (int pos = 0; pos < d.S; ++pos) {
+                const double a = (double)pos * freq;
+                tab[((size_t)pos * half + i) * 2] = (float)cos(a);
+                tab[((size_t)pos * half + i) * 2 + 1] = (float)sin(a);
+            }
+        }
+        KD_CUDA(c, cudaMemcpyAsync(c->arena + y.rope, tab.data(), tab.size() * sizeof(float), cudaMemcpyHostToDevice, s));
+        KD_CUDA(c, cudaStreamSynchronize(s));  // the host table is freed on return
+    }
     c->has_weights = true;
     return KD_OK;
 }
@@ -408,6 +428,8 @@ int kd_sync(kd_ctx* c) {
     if (st[0] != 0) {
         c->failed = true;
         const unsigned w = (unsigned)st[1];
+        if (st[0] == (unsigned long long)kStatusToken)
+            return fail(c, KD_ETOKEN, "a token id outside [0, vocab) reached the kernel at step %u", w & 0xff);
         return fail(c, KD_ETIMEOUT, "device wait exceeded its limit (kind %u, cta %u, detail %u)", w >> 24,
                     (w >> 8) & 0xffff, w & 0xff);
     }
@@ -474,6 +496,7 @@ const char* kd_strerror(int code) {
         case KD_ECUDA: return "CUDA runtime error";
         case KD_ETIMEOUT: return "device-side wait exceeded its limit";
         case KD_ESTATE: return "call out of order";
+        case KD_ETOKEN: return "token id outside the vocabulary";
         default: return "unknown error";
     }
 }

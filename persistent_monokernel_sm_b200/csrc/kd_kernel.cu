@@ -94,6 +94,11 @@ __device__ __forceinline__ uint64_t ld_acquire_u64(const unsigned long long* p) 
 __device__ __forceinline__ void red_release_add_u64(unsigned long long* p, uint64_t v) {
     asm volatile("red.release.gpu.global.add.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
+__device__ __forceinline__ unsigned int atom_add_acq_rel_u32(unsigned int* p, unsigned int v) {
+    unsigned int old;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
+}
 __device__ __forceinline__ void consumer_sync() {
     asm volatile("bar.sync 1, %0;" ::"n"(kConsumerThreads) : "memory");
 }
@@ -113,13 +118,17 @@ __device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 
 __device__ __forceinline__ int read_status(const unsigned long long* ctl) {
     return static_cast<int>(*reinterpret_cast<const volatile unsigned long long*>(ctl + kCtlStatus));
 }
-__device__ __noinline__ void raise_timeout(unsigned long long* ctl, int where) {
-    if (atomicCAS(ctl + kCtlStatus, 0ull, (unsigned long long)kStatusTimeout) == 0ull)
+// The first error of a launch wins: its code goes to the status word, its place to kCtlWhere.
+__device__ __noinline__ void raise_status(unsigned long long* ctl, int code, int where) {
+    if (atomicCAS(ctl + kCtlStatus, 0ull, (unsigned long long)code) == 0ull)
         atomicExch(ctl + kCtlWhere, (unsigned long long)where);
 }
+__device__ __forceinline__ void raise_timeout(unsigned long long* ctl, int where) {
+    raise_status(ctl, kStatusTimeout, where);
+}
 
-// Where a wait gave up: (what << 24) | (cta << 8) | detail.
-enum { kWhereFull = 1, kWhereEmpty = 2, kWhereGrid = 3, kWhereKv = 4 };
+// Where a wait gave up or an input was refused: (what << 24) | (cta << 8) | detail.
+enum { kWhereFull = 1, kWhereEmpty = 2, kWhereGrid = 3, kWhereKv = 4, kWhereToken = 5 };
 __device__ __forceinline__ int where_code(int what, int detail) {
     return (what << 24) | ((int)blockIdx.x << 8) | (detail & 0xff);
 }
@@ -313,18 +322,16 @@ __device__ __forceinline__ bool mbar_wait_hint(uint32_t a, uint32_t parity) {
     return ok != 0;
 }
 
-__device__ bool wait_full(const Smem& sm, const Ring& rg, const Params& P, unsigned long long* ctl,
-                          unsigned long long* waited = nullptr) {
+// `waited` accumulates the cycles spent here (read by the trace only).
+__device__ __forceinline__ bool wait_full(const Smem& sm, const Ring& rg, const Params& P, unsigned long long* ctl,
+                                          unsigned long long& waited) {
     const uint32_t a = smem_u32(&sm.full[rg.slot]);
+    if (__all_sync(0xffffffffu, mbar_try_wait(a, rg.phase))) return true;
     const long long c0 = clock64();
-    if (__all_sync(0xffffffffu, mbar_try_wait(a, rg.phase))) {
-        if (waited) *waited += (unsigned long long)(clock64() - c0);
-        return true;
-    }
     const uint64_t t0 = globaltimer();
     for (;;) {
         if (__all_sync(0xffffffffu, mbar_wait_hint(a, rg.phase))) {
-            if (waited) *waited += (unsigned long long)(clock64() - c0);
+            waited += (unsigned long long)(clock64() - c0);
             return true;
         }
         int bad = 0;
@@ -345,7 +352,7 @@ __device__ bool wait_full(const Smem& sm, const Ring& rg, const Params& P, unsig
 // `local_ok` is false in a warp whose wait gave up; the result is the same for every
 // consumer thread of the CTA, and false in every CTA once any wait anywhere has given up
 // (the device status word is re-read after the barrier completes).
-__device__ bool grid_sync(const Smem& sm, long long& epoch, uint64_t base, const Params& P,
+__device__ __forceinline__ bool grid_sync(const Smem& sm, long long& epoch, uint64_t base, const Params& P,
                           unsigned long long* ctl, bool local_ok, Tracer& tr) {
     // every consumer warp's writes of this phase are done; did every warp succeed?
     const bool cta_ok = consumer_sync_and(local_ok);
@@ -386,7 +393,7 @@ __device__ bool grid_sync(const Smem& sm, long long& epoch, uint64_t base, const
 
 // xs <- x * rsqrt(mean(x^2) + eps) * g in split layout. src_f32 (global, written during
 // the launch) or src_bf16 (an embedding row, read-only).
-__device__ void load_rmsnorm(const Smem& sm, const float* src_f32, const __nv_bfloat16* src_bf16,
+__device__ __forceinline__ void load_rmsnorm(const Smem& sm, const float* src_f32, const __nv_bfloat16* src_bf16,
                              const __nv_bfloat16* gain, int K, float eps) {
     const int tid = threadIdx.x;
     float ss = 0.f;
@@ -424,7 +431,7 @@ __device__ void load_rmsnorm(const Smem& sm, const float* src_f32, const __nv_bf
 }
 
 // xs <- silu(gate) * up for the F interleaved (gate, up) pairs of the raw projection.
-__device__ void load_swiglu(const Smem& sm, const float* gu, int F) {
+__device__ __forceinline__ void load_swiglu(const Smem& sm, const float* gu, int F) {
 #pragma unroll 4
     for (int k = threadIdx.x * 4; k < F; k += kConsumerThreads * 4) {
         const float4 p = __ldcg(reinterpret_cast<const float4*>(gu + 2 * k));
@@ -439,7 +446,7 @@ __device__ void load_swiglu(const Smem& sm, const float* gu, int F) {
     consumer_sync();
 }
 
-__device__ void load_vector(const Smem& sm, const float* src, int K) {
+__device__ __forceinline__ void load_vector(const Smem& sm, const float* src, int K) {
 #pragma unroll 4
     for (int k = threadIdx.x * 4; k < K; k += kConsumerThreads * 4)
         *reinterpret_cast<float4*>(&sm.xs[xs_index(k, K)]) = __ldcg(reinterpret_cast<const float4*>(src + k));
@@ -495,10 +502,14 @@ __device__ __forceinline__ void row_out(const Params& P, const Smem& sm, int pha
 // A wait that gives up marks `ok` false and the warp skips the work of the remaining
 // stages, but it still reaches every named barrier; the next grid barrier then reports
 // the failure to the whole CTA at once.
-__device__ __noinline__ void run_gemv(const Params& P, const Smem& sm_ref, unsigned long long* ctl, int phase, int l,
-                                      Ring& rg_ref, StepCtx& sc_ref, bool& ok_ref, Tracer& tr) {
-    // A separate function (its own register allocation) working on register copies of the
-    // caller's state, written back at the end.
+//
+// NCL > 0: every warp's slice is exactly NCL chunks per lane, so the chunk loop has no
+// per-lane bounds test and its shared-memory addresses are one base plus constants (this
+// is the case for every shape whose reduction length is a multiple of 256 x slices). NCL = 0
+// is the general case (any multiple of 64), with a per-chunk test.
+template <int NCL>
+__device__ __forceinline__ void run_gemv_t(const Params& P, const Smem& sm_ref, unsigned long long* ctl, int phase, int l,
+                                        Ring& rg_ref, StepCtx& sc_ref, bool& ok_ref, Tracer& tr) {
     const Smem sm = sm_ref;
     Ring rg = rg_ref;
     StepCtx sc = sc_ref;
@@ -514,17 +525,19 @@ __device__ __noinline__ void run_gemv(const Params& P, const Smem& sm_ref, unsig
     const int c0 = nch * ks / KS, c1 = nch * (ks + 1) / KS;  // at most 32 * kMaxChunks chunks
     const size_t rowb = (size_t)g.K * 2;
     const int own0 = (int)((long long)P.dm.d * blockIdx.x / P.nb);
-    unsigned long long* waited = threadIdx.x == 0 ? &tr.waited : nullptr;
+    unsigned long long& waited = tr.waited;
 
     // this lane's activation chunks: c = c0 + lane + 32 i
-    float xr[kMaxChunks][8];
+    constexpr int NX = NCL > 0 ? NCL : kMaxChunks;
+    float xr[NX][8];
     const float4* xlo = reinterpret_cast<const float4*>(sm.xs);
     const float4* xhi = reinterpret_cast<const float4*>(sm.xs + (g.K >> 1));
 #pragma unroll
-    for (int i = 0; i < kMaxChunks; ++i) {
+    for (int i = 0; i < NX; ++i) {
         const int c = c0 + lane + 32 * i;
-        const float4 a = c < c1 ? xlo[c] : make_float4(0.f, 0.f, 0.f, 0.f);
-        const float4 b = c < c1 ? xhi[c] : make_float4(0.f, 0.f, 0.f, 0.f);
+        const bool in = NCL > 0 || c < c1;
+        const float4 a = in ? xlo[c] : make_float4(0.f, 0.f, 0.f, 0.f);
+        const float4 b = in ? xhi[c] : make_float4(0.f, 0.f, 0.f, 0.f);
         xr[i][0] = a.x, xr[i][1] = a.y, xr[i][2] = a.z, xr[i][3] = a.w;
         xr[i][4] = b.x, xr[i][5] = b.y, xr[i][6] = b.z, xr[i][7] = b.w;
     }
@@ -533,11 +546,11 @@ __device__ __noinline__ void run_gemv(const Params& P, const Smem& sm_ref, unsig
     // two cross-lane reductions interleave, and the per-stage bookkeeping is paid once per pair.
     auto dot_row = [&](const uint8_t* wrow, float& s) {
         float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+        const uint8_t* wl = wrow + (c0 + lane) * 16;  // this lane's first chunk; then +512 B each
 #pragma unroll
-        for (int i = 0; i < kMaxChunks; ++i) {
-            const int c = c0 + lane + 32 * i;
-            if (c < c1) {
-                const uint4 w = *reinterpret_cast<const uint4*>(wrow + (size_t)c * 16);
+        for (int i = 0; i < NX; ++i) {
+            if (NCL > 0 || c0 + lane + 32 * i < c1) {
+                const uint4 w = *reinterpret_cast<const uint4*>(wl + i * 512);
                 a0 = fmaf(bf_lo(w.x), xr[i][0], a0);
                 a1 = fmaf(bf_hi(w.x), xr[i][1], a1);
                 a2 = fmaf(bf_lo(w.y), xr[i][2], a2);
@@ -635,6 +648,28 @@ __device__ __noinline__ void run_gemv(const Params& P, const Smem& sm_ref, unsig
     }
 }
 
+// Chunks (8 elements) per lane of every warp's slice when that count is exact, else 0.
+__device__ __forceinline__ int gemv_exact_chunks(int K, int R) {
+    const int KS = kGroupWarps / R, nch = K >> 3;
+    return nch % (32 * KS) == 0 && nch / (32 * KS) <= kMaxChunks ? nch / (32 * KS) : 0;
+}
+
+__device__ __forceinline__ void run_gemv(const Params& P, const Smem& sm, unsigned long long* ctl, int phase, int l,
+                                      Ring& rg, StepCtx& sc, bool& ok, Tracer& tr) {
+    const Gemv g = gemv_geom(P, phase, l, blockIdx.x);
+    switch (gemv_exact_chunks(g.K, g.R)) {
+        case 1: run_gemv_t<1>(P, sm, ctl, phase, l, rg, sc, ok, tr); break;
+        case 2: run_gemv_t<2>(P, sm, ctl, phase, l, rg, sc, ok, tr); break;
+        case 3: run_gemv_t<3>(P, sm, ctl, phase, l, rg, sc, ok, tr); break;
+        case 4: run_gemv_t<4>(P, sm, ctl, phase, l, rg, sc, ok, tr); break;
+        case 5: run_gemv_t<5>(P, sm, ctl, phase, l, rg, sc, ok, tr); break;
+        case 6: run_gemv_t<6>(P, sm, ctl, phase, l, rg, sc, ok, tr); break;
+        case 7: run_gemv_t<7>(P, sm, ctl, phase, l, rg, sc, ok, tr); break;
+        case 8: run_gemv_t<8>(P, sm, ctl, phase, l, rg, sc, ok, tr); break;
+        default: run_gemv_t<0>(P, sm, ctl, phase, l, rg, sc, ok, tr); break;
+    }
+}
+
 // Loads that read either the shared-memory ring or, for the current position, the cache
 // itself (written during this launch: L2 only).
 __device__ __forceinline__ uint4 ld16(const __nv_bfloat16* p, bool global) {
@@ -657,10 +692,11 @@ __device__ __forceinline__ void ld_v(const __nv_bfloat16* p, bool global, float 
 // all lanes accumulate the 8 V rows (each lane hd/32 output dims). States of the warps are
 // merged per CTA; the last CTA of a kv head to finish combines all pieces.
 // GMAX >= the number of q heads per kv head (2, 4 or 8).
+constexpr int kCombineBatch = 12;  // pieces whose records one combining thread loads at once
 template <int HD, int GMAX>
-__device__ __noinline__ void run_attention(const Params& P, const Smem& sm_ref, unsigned long long* ctl, int l,
+__device__ __forceinline__ void run_attention(const Params& P, const Smem& sm_ref, unsigned long long* ctl, int l,
                                           Ring& rg_ref, StepCtx& sc_ref, bool& ok_ref, Tracer& tr) {
-    const Smem sm = sm_ref;  // register copies (see run_gemv_t)
+    const Smem sm = sm_ref;
     const StepCtx sc = sc_ref;
     Ring rg = rg_ref;
     bool ok = ok_ref;
@@ -675,38 +711,49 @@ __device__ __noinline__ void run_attention(const Params& P, const Smem& sm_ref, 
     const float qscale = 1.4426950408889634f / sqrtf((float)HD);  // log2(e) / sqrt(hd)
     // The Q/K/V projections arrive raw, q and k rows in RoPE-pair order (row 2i = dim i,
     // row 2i + 1 = dim i + hd/2). Rotate this group's q heads at position p while loading.
+    // The piece that holds position p also appends that position's K (rotated) and V to the
+    // cache, rounded to bf16, and keeps a copy for its own pass below. Every load of this
+    // prologue is issued before any store (one L2 round trip): at most 2 q pairs per thread
+    // (r * HD / 2 <= 512), and one K and one V pair for threads below HD / 2.
     const float* raw = reinterpret_cast<const float*>(P.arena + P.lay.qkv);
     const float* qg = raw + (size_t)at.g * r * HD;
-    for (int t = tid; t < r * HD / 2; t += kConsumerThreads) {
-        const int hh = t / (HD / 2), i = t % (HD / 2);
-        const float a = __ldcg(qg + hh * HD + 2 * i), b = __ldcg(qg + hh * HD + 2 * i + 1);
-        const float2 cs = sm.rope[i];
-        sm.qs[hh * HD + i] = (a * cs.x - b * cs.y) * qscale;
-        sm.qs[hh * HD + i + HD / 2] = (b * cs.x + a * cs.y) * qscale;
-    }
-    // The piece that holds position p appends that position's K (rotated) and V to the
-    // cache, rounded to bf16, and keeps a copy for its own pass below.
     const bool has_current = at.b > sc.p;
-    if (has_current) {
+    const bool kv_lane = has_current && tid < HD / 2;
+    float2 qv[2], kv2, vv2;
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+        const int t = tid + u * kConsumerThreads;
+        if (t < r * HD / 2) qv[u] = __ldcg(reinterpret_cast<const float2*>(qg + (t / (HD / 2)) * HD + 2 * (t % (HD / 2))));
+    }
+    if (kv_lane) {
+        kv2 = __ldcg(reinterpret_cast<const float2*>(raw + dm.qd + (size_t)at.g * HD + 2 * tid));
+        vv2 = __ldcg(reinterpret_cast<const float2*>(raw + dm.qd + dm.kvd + (size_t)at.g * HD + 2 * tid));
+    }
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+        const int t = tid + u * kConsumerThreads;
+        if (t < r * HD / 2) {
+            const int hh = t / (HD / 2), i = t % (HD / 2);
+            const float2 cs = sm.rope[i];
+            sm.qs[hh * HD + i] = (qv[u].x * cs.x - qv[u].y * cs.y) * qscale;
+            sm.qs[hh * HD + i + HD / 2] = (qv[u].y * cs.x + qv[u].x * cs.y) * qscale;
+        }
+    }
+    if (kv_lane) {
+        const int i = tid;
         const size_t off = (((size_t)l * dm.Hkv + at.g) * dm.S + sc.p) * HD;
         __nv_bfloat16* kc = reinterpret_cast<__nv_bfloat16*>(const_cast<uint8_t*>(P.arena) + P.lay.kcache) + off;
         __nv_bfloat16* vc = reinterpret_cast<__nv_bfloat16*>(const_cast<uint8_t*>(P.arena) + P.lay.vcache) + off;
-        const float* kr = raw + dm.qd + (size_t)at.g * HD;
-        const float* vr = raw + dm.qd + dm.kvd + (size_t)at.g * HD;
-        for (int i = tid; i < HD / 2; i += kConsumerThreads) {
-            const float a = __ldcg(kr + 2 * i), b = __ldcg(kr + 2 * i + 1);
-            const float2 cs = sm.rope[i];
-            const __nv_bfloat16 k0 = __float2bfloat16_rn(a * cs.x - b * cs.y);
-            const __nv_bfloat16 k1 = __float2bfloat16_rn(b * cs.x + a * cs.y);
-            kc[i] = k0, kc[i + HD / 2] = k1;
-            sm.kvcur[i] = k0, sm.kvcur[i + HD / 2] = k1;
-            const __nv_bfloat16 v0 = __float2bfloat16_rn(__ldcg(vr + 2 * i));
-            const __nv_bfloat16 v1 = __float2bfloat16_rn(__ldcg(vr + 2 * i + 1));
-            vc[2 * i] = v0, vc[2 * i + 1] = v1;
-            sm.kvcur[HD + 2 * i] = v0, sm.kvcur[HD + 2 * i + 1] = v1;
-        }
-        fence_proxy_async_global();  // later bulk copies (async proxy) read these rows
+        const float2 cs = sm.rope[i];
+        const __nv_bfloat16 k0 = __float2bfloat16_rn(kv2.x * cs.x - kv2.y * cs.y);
+        const __nv_bfloat16 k1 = __float2bfloat16_rn(kv2.y * cs.x + kv2.x * cs.y);
+        kc[i] = k0, kc[i + HD / 2] = k1;
+        sm.kvcur[i] = k0, sm.kvcur[i + HD / 2] = k1;
+        const __nv_bfloat162 v01 = __floats2bfloat162_rn(vv2.x, vv2.y);
+        *reinterpret_cast<__nv_bfloat162*>(vc + 2 * i) = v01;
+        *reinterpret_cast<__nv_bfloat162*>(&sm.kvcur[HD + 2 * i]) = v01;
     }
+    if (has_current) fence_proxy_async_global();  // later bulk copies (async proxy) read these rows
     consumer_sync();
     if (tid == 0) tr.mark(4);
 
@@ -807,7 +854,7 @@ __device__ __noinline__ void run_attention(const Params& P, const Smem& sm_ref, 
     // most 16 (two blocks of one pass) with hd 64.
     const int nst = attn_stages(P, at);
     const int group = warp / kGroupWarps, gw = warp % kGroupWarps;
-    unsigned long long* waited = tid == 0 ? &tr.waited : nullptr;
+    unsigned long long& waited = tr.waited;
     for (int j = 0; j < nst; ++j, rg.advance(P.ns)) {
         if (rg.slot % kGroups != group || !ok) continue;  // group g: slots g mod kGroups
         if (!wait_full(sm, rg, P, ctl, waited)) {
@@ -863,53 +910,50 @@ __device__ __noinline__ void run_attention(const Params& P, const Smem& sm_ref, 
     }
     consumer_sync();
     if (tid == 0) {
-        __threadfence();
+        // one acquire-release add: publishes this CTA's partial records (ordered before it by
+        // the barrier above) and, for the last piece to arrive, makes everyone else's visible
         unsigned int* cnt = reinterpret_cast<unsigned int*>(ctl + kCtlHead + 16 * at.g);
-        const unsigned int old = atomicAdd(cnt, 1u);
+        const unsigned int old = atom_add_acq_rel_u32(cnt, 1u);
         sm.flag[1] = ((old + 1u) % (unsigned)A) == 0u;
-        __threadfence();
     }
     consumer_sync();
     if (sm.flag[1]) {  // last piece of this kv head to finish: combine all pieces
+        // Each thread owns output (h, dd) and reads (m_i, l_i, acc_i[dd]) of the pieces in
+        // batches of kCombineBatch, all loads of a batch in flight together, folding each
+        // batch in with the usual max-rescaled sum (pieces in ascending order).
         const float* hp = part + (size_t)at.g * A * r * rec;
-        float* fw = sm.xs;                    // [h][A] piece weights
-        float* invl = sm.xs + kMaxGroup * A;  // [h]
-        if (warp < r) {  // warp h: the weights 2^(m_i - M) of head h's pieces and 1 / L
-            const int h = warp;
-            float M = -INFINITY;
-            for (int i = lane; i < A; i += 32) M = fmaxf(M, __ldcg(hp + ((size_t)i * r + h) * rec));
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-            float L = 0.f;
-            for (int i = lane; i < A; i += 32) {
-                const float* pr = hp + ((size_t)i * r + h) * rec;
-                const float mi = __ldcg(pr);
-                const float f = mi == -INFINITY ? 0.f : exp2f(mi - M);
-                fw[h * A + i] = f;
-                L = fmaf(__ldcg(pr + 1), f, L);
-            }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
-            if (lane == 0) invl[h] = 1.0f / L;
-        }
-        consumer_sync();
         float* og = reinterpret_cast<float*>(const_cast<uint8_t*>(P.arena) + P.lay.o) + (size_t)at.g * r * HD;
+        const size_t stride = (size_t)r * rec;
         for (int idx = tid; idx < r * HD; idx += kConsumerThreads) {
             const int h = idx / HD, dd = idx % HD;
-            const float* src = hp + (size_t)h * rec + 2 + dd;
-            const size_t stride = (size_t)r * rec;
-            float o0 = 0.f, o1 = 0.f, o2 = 0.f, o3 = 0.f;
-            int i = 0;
-            for (; i + 4 <= A; i += 4) {  // four independent loads in flight
-                const float a0 = __ldcg(src + (size_t)i * stride), a1 = __ldcg(src + (size_t)(i + 1) * stride);
-                const float a2 = __ldcg(src + (size_t)(i + 2) * stride), a3 = __ldcg(src + (size_t)(i + 3) * stride);
-                o0 = fmaf(a0, fw[h * A + i], o0);
-                o1 = fmaf(a1, fw[h * A + i + 1], o1);
-                o2 = fmaf(a2, fw[h * A + i + 2], o2);
-                o3 = fmaf(a3, fw[h * A + i + 3], o3);
+            const float* src = hp + (size_t)h * rec;
+            float M = -INFINITY, L = 0.f, o = 0.f;
+            for (int i0 = 0; i0 < A; i0 += kCombineBatch) {
+                float mi[kCombineBatch], li[kCombineBatch], ai[kCombineBatch];
+#pragma unroll
+                for (int k = 0; k < kCombineBatch; ++k) {
+                    mi[k] = -INFINITY, li[k] = 0.f, ai[k] = 0.f;  // pieces past A weigh nothing
+                    if (i0 + k < A) {
+                        const float* pr = src + (size_t)(i0 + k) * stride;
+                        mi[k] = __ldcg(pr), li[k] = __ldcg(pr + 1), ai[k] = __ldcg(pr + 2 + dd);
+                    }
+                }
+                float Mb = M;
+#pragma unroll
+                for (int k = 0; k < kCombineBatch; ++k) Mb = fmaxf(Mb, mi[k]);
+                if (Mb != -INFINITY) {  // else no position in these pieces yet
+                    const float c = exp2f(M - Mb);  // 0 when M is still -inf
+                    L *= c, o *= c;
+#pragma unroll
+                    for (int k = 0; k < kCombineBatch; ++k) {
+                        const float f = exp2f(mi[k] - Mb);  // 0 for an empty or absent piece
+                        L = fmaf(li[k], f, L);
+                        o = fmaf(ai[k], f, o);
+                    }
+                    M = Mb;
+                }
             }
-            for (; i < A; ++i) o0 = fmaf(__ldcg(src + (size_t)i * stride), fw[h * A + i], o0);
-            __stcg(og + (size_t)h * HD + dd, ((o0 + o1) + (o2 + o3)) * invl[h]);
+            __stcg(og + (size_t)h * HD + dd, o / L);
         }
         if (tid == 0) tr.mark(7);
     }
@@ -1123,8 +1167,10 @@ struct Producer {
             ok = issue(ld);
             ld.next(P);
         }
-        if (!ok) {
-            // unwinding: let every copy already issued land before the CTA exits
+        // Let every copy already issued land before the CTA exits: when the consumers have
+        // stopped early (a refused token, a wait that gave up) nobody else waits for them.
+        // On a normal run these stages were consumed already and each test passes at once.
+        {
             const int first = k > P.ns ? k - P.ns : 0;
             for (int kk = first; kk < k; ++kk) {
                 const uint32_t a = smem_u32(&sm.full[kk % P.ns]);
@@ -1144,6 +1190,9 @@ struct Producer {
 
 // ------------------------------------------------------------------ the kernel
 
+// One instantiation per attention shape (head dim, q heads per kv head rounded up to 2, 4
+// or 8), so the fully inlined kernel holds one attention body and its registers.
+template <int HD, int GMAX>
 __global__ void __launch_bounds__(kThreads, 1) monokernel(const __grid_constant__ Params P) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const Smem sm = carve(P, smem_raw);
@@ -1208,16 +1257,22 @@ __global__ void __launch_bounds__(kThreads, 1) monokernel(const __grid_constant_
                 if (blockIdx.x == 0) P.tokens_out[t - P.n_pending] = tok;
             }
             if (blockIdx.x == 0) ctl[kCtlArgmax + 16 * ((t + 1) % 3)] = 0ull;
+            // A token id outside the vocabulary (a bad pending input) stops the launch before
+            // the embedding row is read. Every CTA reads the same id, so all of them stop here.
+            if ((unsigned)tok >= (unsigned)dm.V) {
+                raise_status(ctl, kStatusToken, where_code(kWhereToken, t));
+                tok = -1;
+            }
             sm.flag[2] = tok;
         }
-        if (tid < dm.hd / 2) {
-            const double freq = pow((double)dm.theta, -2.0 * (double)tid / (double)dm.hd);
-            double s, c;
-            sincos((double)sc.p * freq, &s, &c);
-            sm.rope[tid] = make_float2((float)c, (float)s);
-        }
+        if (tid < dm.hd / 2)  // this position's RoPE row (cos, sin per pair)
+            sm.rope[tid] = __ldg(reinterpret_cast<const float2*>(P.arena + P.lay.rope) + (size_t)sc.p * (dm.hd / 2) + tid);
         consumer_sync();
         const int tok = sm.flag[2];
+        if (tok < 0) {
+            ok = false;
+            break;
+        }
         const __nv_bfloat16* erow = embed + (size_t)tok * dm.d;
         for (int i = own0 + tid; i < own1; i += kConsumerThreads) {
             const float v = __bfloat162float(erow[i]);
@@ -1225,54 +1280,40 @@ __global__ void __launch_bounds__(kThreads, 1) monokernel(const __grid_constant_
             __stcg(xg + i, v);
         }
 
-        for (int l = 0; l < dm.L && ok; ++l) {
+        // The step's phases in order: per layer QKV, ATT, O, GU, D, then the LM head if this
+        // step's logits are needed. One loop with one call site per phase kind keeps the
+        // (fully inlined) kernel's code and register allocation to one copy of each.
+        const int nphase = 5 * dm.L + (step_has_head(P, t) ? 1 : 0);
+        for (int q = 0; q < nphase; ++q) {
+            const int l = q / 5 < dm.L ? q / 5 : 0;
+            const int ph = q / 5 < dm.L ? q % 5 : kLM;
             sc.l = l;
             const uint8_t* lb = P.arena + P.lay.layer0 + (size_t)l * P.lay.layer_stride;
-            const __nv_bfloat16* gattn = reinterpret_cast<const __nv_bfloat16*>(lb + P.lay.l_attn_norm);
-            const __nv_bfloat16* gffn = reinterpret_cast<const __nv_bfloat16*>(lb + P.lay.l_ffn_norm);
-            // attention block
-            if (l == 0) load_rmsnorm(sm, nullptr, erow, gattn, dm.d, dm.eps);
-            else load_rmsnorm(sm, xg, nullptr, gattn, dm.d, dm.eps);
-            if (tid == 0) tr.mark(1);
-            run_gemv(P, sm, ctl, kQKV, l, rg, sc, ok, tr);
-            if (!(ok = grid_sync(sm, epoch, base, P, ctl, ok, tr))) break;
-            if (tid == 0) tr.mark(1);
-            if (dm.hd == 128) {
-                if (dm.r <= 2) run_attention<128, 2>(P, sm, ctl, l, rg, sc, ok, tr);
-                else if (dm.r <= 4) run_attention<128, 4>(P, sm, ctl, l, rg, sc, ok, tr);
-                else run_attention<128, 8>(P, sm, ctl, l, rg, sc, ok, tr);
-            } else {
-                if (dm.r <= 2) run_attention<64, 2>(P, sm, ctl, l, rg, sc, ok, tr);
-                else if (dm.r <= 4) run_attention<64, 4>(P, sm, ctl, l, rg, sc, ok, tr);
-                else run_attention<64, 8>(P, sm, ctl, l, rg, sc, ok, tr);
+            // this phase's input vector -> xs
+            if (ph == kO) {
+                load_vector(sm, reinterpret_cast<const float*>(P.arena + P.lay.o), dm.qd);
+            } else if (ph == kD) {
+                load_swiglu(sm, reinterpret_cast<const float*>(P.arena + P.lay.gu), dm.F);
+            } else if (ph != kATT) {
+                const __nv_bfloat16* gain = reinterpret_cast<const __nv_bfloat16*>(
+                    ph == kQKV ? lb + P.lay.l_attn_norm : ph == kGU ? lb + P.lay.l_ffn_norm : P.arena + P.lay.final_norm);
+                const bool from_embed = ph == kQKV && l == 0;
+                load_rmsnorm(sm, from_embed ? nullptr : xg, from_embed ? erow : nullptr, gain, dm.d, dm.eps);
             }
-            if (!(ok = grid_sync(sm, epoch, base, P, ctl, ok, tr))) break;
-            load_vector(sm, reinterpret_cast<const float*>(P.arena + P.lay.o), dm.qd);
             if (tid == 0) tr.mark(1);
-            run_gemv(P, sm, ctl, kO, l, rg, sc, ok, tr);
-            if (!(ok = grid_sync(sm, epoch, base, P, ctl, ok, tr))) break;
-            // feed-forward block
-            load_rmsnorm(sm, xg, nullptr, gffn, dm.d, dm.eps);
-            if (tid == 0) tr.mark(1);
-            run_gemv(P, sm, ctl, kGU, l, rg, sc, ok, tr);
-            if (!(ok = grid_sync(sm, epoch, base, P, ctl, ok, tr))) break;
-            load_swiglu(sm, reinterpret_cast<const float*>(P.arena + P.lay.gu), dm.F);
-            if (tid == 0) tr.mark(1);
-            run_gemv(P, sm, ctl, kD, l, rg, sc, ok, tr);
-            if (!(ok = grid_sync(sm, epoch, base, P, ctl, ok, tr))) break;
-        }
-        if (!ok) break;
-        if (step_has_head(P, t)) {
-            load_rmsnorm(sm, xg, nullptr, reinterpret_cast<const __nv_bfloat16*>(P.arena + P.lay.final_norm),
-                         dm.d, dm.eps);
-            if (tid == 0) tr.mark(1);
-            run_gemv(P, sm, ctl, kLM, 0, rg, sc, ok, tr);
-            if ((tid & 31) == 0) sm.best[tid >> 5] = sc.lm_best;
-            consumer_sync();
-            if (tid == 0 && ok) {
-                unsigned long long b = 0ull;
-                for (int w = 0; w < kConsumerWarps; ++w) b = sm.best[w] > b ? sm.best[w] : b;
-                atomicMax(ctl + kCtlArgmax + 16 * (t % 3), b);
+            if (ph == kATT) {
+                run_attention<HD, GMAX>(P, sm, ctl, l, rg, sc, ok, tr);
+            } else {
+                run_gemv(P, sm, ctl, ph, l, rg, sc, ok, tr);
+            }
+            if (ph == kLM) {
+                if ((tid & 31) == 0) sm.best[tid >> 5] = sc.lm_best;
+                consumer_sync();
+                if (tid == 0 && ok) {
+                    unsigned long long b = 0ull;
+                    for (int w = 0; w < kConsumerWarps; ++w) b = sm.best[w] > b ? sm.best[w] : b;
+                    atomicMax(ctl + kCtlArgmax + 16 * (t % 3), b);
+                }
             }
             if (!(ok = grid_sync(sm, epoch, base, P, ctl, ok, tr))) break;
         }
@@ -1291,16 +1332,28 @@ __global__ void __launch_bounds__(kThreads, 1) monokernel(const __grid_constant_
 
 // ------------------------------------------------------------------ host-side launch
 
-int monokernel_occupancy(int smem_bytes, int* blocks_per_sm) {
-    cudaError_t e = cudaFuncSetAttribute(monokernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
+static const void* kernel_for(int hd, int r) {
+    if (hd == 128) {
+        if (r <= 2) return (const void*)monokernel<128, 2>;
+        if (r <= 4) return (const void*)monokernel<128, 4>;
+        return (const void*)monokernel<128, 8>;
+    }
+    if (r <= 2) return (const void*)monokernel<64, 2>;
+    if (r <= 4) return (const void*)monokernel<64, 4>;
+    return (const void*)monokernel<64, 8>;
+}
+
+int monokernel_occupancy(int hd, int r, int smem_bytes, int* blocks_per_sm) {
+    const void* k = kernel_for(hd, r);
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
     if (e != cudaSuccess) return (int)e;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, monokernel, kThreads, smem_bytes);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, k, kThreads, smem_bytes);
     return (int)e;
 }
 
 void launch_decode(const Params& p, void* stream, int smem_bytes, int* err) {
     void* args[] = {const_cast<Params*>(&p)};
-    cudaError_t e = cudaLaunchCooperativeKernel((const void*)monokernel, dim3(p.nb), dim3(kThreads), args,
+    cudaError_t e = cudaLaunchCooperativeKernel(kernel_for(p.dm.hd, p.dm.r), dim3(p.nb), dim3(kThreads), args,
                                                 (size_t)smem_bytes, (cudaStream_t)stream);
     *err = (int)e;
 }

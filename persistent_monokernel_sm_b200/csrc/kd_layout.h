@@ -30,7 +30,8 @@ constexpr int kCtlArgmax = 32;             // 3 argmax slots at kCtlArgmax + 16*
 constexpr int kCtlHead = 96;               // split-K arrival counters at kCtlHead + 16*g
 constexpr int kCtlWords = kCtlHead + 16 * kMaxKvHeads;
 
-constexpr int kStatusTimeout = 1;
+constexpr int kStatusTimeout = 1;  // a device-side wait exceeded its limit
+constexpr int kStatusToken = 2;    // a token id outside [0, vocab) reached the kernel
 
 struct Dims {
     int L, d, Hq, Hkv, hd, F, V, S;  // S = max_seq
@@ -44,6 +45,7 @@ struct Layout {
     size_t embed, lm_head, final_norm;
     size_t layer0, layer_stride;
     size_t l_attn_norm, l_ffn_norm, l_wqkv, l_wo, l_wgu, l_wd;  // within a layer block
+    size_t rope;                                                  // [S][hd/2] float2 (cos, sin)
     size_t kcache, vcache;                                        // [L][Hkv][S][hd] bf16
     size_t x, qkv, o, gu, part;                                   // fp32 scratch
     size_t ctl, tokens_in, tokens_out;
@@ -113,6 +115,6 @@ struct kd_ctx_view {
     bool has_weights;
 };
 int monokernel_smem_bytes(const Params& p);
-int monokernel_occupancy(int smem_bytes, int* blocks_per_sm);
+int monokernel_occupancy(int hd, int r, int smem_bytes, int* blocks_per_sm);
 
 }  // namespace kd

@@ -141,6 +141,8 @@ extern "C" int kd_decode_noalloc(kd_ctx* ctx, const int32_t* d_tokens, int32_t n
                              (cudaStream_t)v.stream)) != cudaSuccess ||
         (e = cudaStreamSynchronize((cudaStream_t)v.stream)) != cudaSuccess)
         return kd_internal_fail(ctx, KD_ECUDA, cudaGetErrorString(e));
+    if (status == (unsigned long long)kStatusToken)
+        return kd_internal_fail(ctx, KD_ETOKEN, "kd_decode_noalloc: a token id outside [0, vocab) reached the kernel");
     if (status != 0) return kd_internal_fail(ctx, KD_ETIMEOUT, "kd_decode_noalloc: a device-side wait exceeded its limit");
     return KD_OK;
 }

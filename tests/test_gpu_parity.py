@@ -159,6 +159,32 @@ def test_capacity_is_checked_before_launch(kd):
     assert dec.info().launches == before
 
 
+def test_token_outside_vocab_stops_the_launch(kd):
+    """A pending id outside [0, vocab) is refused by the kernel's own range check before any
+    embedding row is read: kd_sync reports KD_ETOKEN, and after kd_reset the handle decodes
+    exactly as before."""
+    w = synth.get("tiny")
+    W = weights_for("tiny")
+    prompt = synth.make_prompt(w).numpy()
+    dec = make_decoder(kd, w, W)
+    dec.reset(prompt, 0)
+    ref, _ = dec.decode(8)
+    dec.sync()
+    ref = ref.cpu().numpy().copy()
+    for bad in (w.vocab, -1):
+        dec.reset(np.concatenate([prompt[:3], [bad], prompt[3:]]).astype(np.int32), 0)
+        dec.decode(4)
+        with pytest.raises(kd.KdError) as e:
+            dec.sync()
+        assert e.value.code == -8
+        with pytest.raises(kd.KdError):
+            dec.decode(1)  # refused until reset
+    dec.reset(prompt, 0)
+    again, _ = dec.decode(8)
+    dec.sync()
+    assert np.array_equal(again.cpu().numpy(), ref)
+
+
 # ------------------------------------------------------------------ 0.5B: every step
 
 def test_half_billion_forced_and_greedy(kd):
