@@ -78,7 +78,7 @@ Layout make_layout(const Dims& d) {
     y.x = take(D * 4);
     y.qkv = take((size_t)d.qkv_rows * 4);  // raw q/k/v projections (repacked row order)
     y.o = take((size_t)d.qd * 4);
-    y.gu = take((size_t)2 * d.F * 4);  // raw gate/up projections, interleaved
+    y.gu = take((size_t)d.F * 4);  // FFN hidden vector silu(gate) * up
     y.part = take((size_t)kMaxGrid * d.r * (d.hd + 2) * 4);
     y.ctl = take((size_t)kCtlWords * 8);
     y.tokens_in = take((size_t)d.S * 4);

@@ -359,7 +359,10 @@ __device__ __forceinline__ bool grid_sync(const Smem& sm, long long& epoch, uint
     if (threadIdx.x == 0) tr.mark(2);
     if (threadIdx.x == 0 && !cta_ok) sm.flag[0] = 0;
     if (threadIdx.x == 0 && cta_ok) {
-        __threadfence();
+        // The release add publishes every consumer thread's writes of this phase (ordered
+        // before it by the CTA barrier above); the acquire poll below makes all CTAs'
+        // writes visible to this thread, and the CTA barrier after it to the others. Loads
+        // of data written during the launch bypass L1 (ld.global.cg), so no fence is needed.
         red_release_add_u64(ctl + kCtlBar, 1ull);
         const uint64_t target = base + (uint64_t)(epoch + 1) * (uint64_t)P.nb;
         int ok = 1;
@@ -377,7 +380,6 @@ __device__ __forceinline__ bool grid_sync(const Smem& sm, long long& epoch, uint
                 }
             }
         }
-        __threadfence();
         if (ok && read_status(ctl) != 0) ok = 0;
         sm.flag[0] = ok;
         tr.mark(3);
@@ -390,6 +392,13 @@ __device__ __forceinline__ bool grid_sync(const Smem& sm, long long& epoch, uint
 }
 
 // ------------------------------------------------------------------ activation loads
+
+// Shared-memory store in asm: the compiler then does not treat it as a possible write to a
+// global source, and may keep later iterations' global loads ahead of it (the asm stays
+// ordered with the barriers, also volatile asm).
+__device__ __forceinline__ void sts128(float* p, float4 v) {
+    asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(smem_u32(p)), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w));
+}
 
 // xs <- x * rsqrt(mean(x^2) + eps) * g in split layout. src_f32 (global, written during
 // the launch) or src_bf16 (an embedding row, read-only).
@@ -407,7 +416,7 @@ __device__ __forceinline__ void load_rmsnorm(const Smem& sm, const float* src_f3
             v = make_float4(bf_lo(w.x), bf_hi(w.x), bf_lo(w.y), bf_hi(w.y));
         }
         ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
-        *reinterpret_cast<float4*>(&sm.xs[xs_index(k, K)]) = v;
+        sts128(&sm.xs[xs_index(k, K)], v);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
@@ -430,26 +439,11 @@ __device__ __forceinline__ void load_rmsnorm(const Smem& sm, const float* src_f3
     consumer_sync();
 }
 
-// xs <- silu(gate) * up for the F interleaved (gate, up) pairs of the raw projection.
-__device__ __forceinline__ void load_swiglu(const Smem& sm, const float* gu, int F) {
-#pragma unroll 4
-    for (int k = threadIdx.x * 4; k < F; k += kConsumerThreads * 4) {
-        const float4 p = __ldcg(reinterpret_cast<const float4*>(gu + 2 * k));
-        const float4 q = __ldcg(reinterpret_cast<const float4*>(gu + 2 * k + 4));
-        float4 h;
-        h.x = p.x / (1.0f + expf(-p.x)) * p.y;
-        h.y = p.z / (1.0f + expf(-p.z)) * p.w;
-        h.z = q.x / (1.0f + expf(-q.x)) * q.y;
-        h.w = q.z / (1.0f + expf(-q.z)) * q.w;
-        *reinterpret_cast<float4*>(&sm.xs[xs_index(k, F)]) = h;
-    }
-    consumer_sync();
-}
-
+// xs <- src (fp32, written during the launch).
 __device__ __forceinline__ void load_vector(const Smem& sm, const float* src, int K) {
 #pragma unroll 4
     for (int k = threadIdx.x * 4; k < K; k += kConsumerThreads * 4)
-        *reinterpret_cast<float4*>(&sm.xs[xs_index(k, K)]) = __ldcg(reinterpret_cast<const float4*>(src + k));
+        sts128(&sm.xs[xs_index(k, K)], __ldcg(reinterpret_cast<const float4*>(src + k)));
     consumer_sync();
 }
 
@@ -470,8 +464,9 @@ struct StepCtx {
 };
 
 // Output of one finished GEMV row (global row index `row`, value y): stored raw for the
-// Q/K/V and gate/up projections (RoPE, the KV-cache append and SwiGLU are applied where the
-// values are consumed), added into the residual for O and down (the CTA owns those rows and
+// Q/K/V projections (RoPE and the KV-cache append are applied where they are consumed),
+// the FFN hidden value silu(gate) * up for a gate/up pair (y is already that value; `row` is
+// the pair's gate row), added into the residual for O and down (the CTA owns those rows and
 // keeps them in shared memory, so no read-back from L2), and for the LM head dumped when
 // requested and folded into this thread's running argmax.
 __device__ __forceinline__ void row_out(const Params& P, const Smem& sm, int phase, int row, float y, StepCtx& sc,
@@ -480,7 +475,7 @@ __device__ __forceinline__ void row_out(const Params& P, const Smem& sm, int pha
     if (phase == kQKV) {
         __stcg(reinterpret_cast<float*>(arena + P.lay.qkv) + row, y);
     } else if (phase == kGU) {
-        __stcg(reinterpret_cast<float*>(arena + P.lay.gu) + row, y);
+        __stcg(reinterpret_cast<float*>(arena + P.lay.gu) + (row >> 1), y);  // hidden value of pair row / 2
     } else if (phase == kO || phase == kD) {
         const float v = sm.xown[row - own0] + y;
         sm.xown[row - own0] = v;
@@ -565,7 +560,7 @@ __device__ __forceinline__ void run_gemv_t(const Params& P, const Smem& sm_ref, 
     };
     // per-stage completion: release the slot and put the row(s) out
     auto finish = [&](const Ring& at_rg, int r0, int n, float part) {
-        if (KS == 1) {  // this warp owns the whole row
+        if (KS == 1 && phase != kGU) {  // this warp owns the whole row
             __syncwarp();
             if (lane == kSyncLane) mbar_arrive(smem_u32(&sm.empty[at_rg.slot]));  // done with the stage
             if (lane == 0 && row < n) row_out(P, sm, phase, r0 + row, part, sc, own0);
@@ -590,7 +585,14 @@ __device__ __forceinline__ void run_gemv_t(const Params& P, const Smem& sm_ref, 
             sm.scnt[at_rg.slot] = 0;
             mbar_arrive(smem_u32(&sm.empty[at_rg.slot]));  // partial sums read: the slot may refill
         }
-        if (lane < n) row_out(P, sm, phase, r0 + lane, tot, sc, own0);
+        if (phase == kGU) {
+            // rows come in (gate, up) pairs, lane 2j holding gate j and lane 2j + 1 up j:
+            // the FFN hidden value silu(gate) * up is formed here, once, for the D phase
+            const float up = __shfl_down_sync(0xffffffffu, tot, 1);
+            if (lane < n && (lane & 1) == 0) row_out(P, sm, phase, r0 + lane, tot / (1.0f + expf(-tot)) * up, sc, own0);
+        } else if (lane < n) {
+            row_out(P, sm, phase, r0 + lane, tot, sc, own0);
+        }
     };
 
     int j = 0;
@@ -621,6 +623,7 @@ __device__ __forceinline__ void run_gemv_t(const Params& P, const Smem& sm_ref, 
             ok = false;
             continue;
         }
+        if (threadIdx.x == 0 && ja == 0) tr.mark(4);  // first stage of the phase ready
         const int ra0 = g.row0 + ja * g.R, na = min(g.R, g.row1 - ra0);
         const int rb0 = g.row0 + jb * g.R, nb = two ? min(g.R, g.row1 - rb0) : 0;
         float pa = 0.f, pb = 0.f;
@@ -634,6 +637,7 @@ __device__ __forceinline__ void run_gemv_t(const Params& P, const Smem& sm_ref, 
         finish(ra, ra0, na, pa);
         if (two) finish(rb, rb0, nb, pb);
     }
+    if (threadIdx.x == 0) tr.mark(5);  // this warp's stages done
     rg_ref = rg;
     ok_ref = ok;
     // LM head: fold the lanes' running argmax into lane 0's (lowest index on ties)
@@ -849,28 +853,53 @@ __device__ __forceinline__ void run_attention(const Params& P, const Smem& sm_re
         }
     };
 
-    // Stages alternate between the two groups (ring-slot parity); within a stage, warp gw of
-    // the group takes positions [n * gw / 8, n * (gw + 1) / 8): at most 8 with hd 128, at
-    // most 16 (two blocks of one pass) with hd 64.
+    // Within a stage, warp gw takes positions [n * gw / 8, n * (gw + 1) / 8): at most 8 with
+    // hd 128, at most 16 (the two blocks of one pass) with hd 64. With hd 128 a warp takes two
+    // stages per pass, one block from each, so each online-softmax update covers 16 positions.
+    static_assert(kGroups == 1, "attention stages assume one consumer group");
     const int nst = attn_stages(P, at);
-    const int group = warp / kGroupWarps, gw = warp % kGroupWarps;
+    const int gw = warp % kGroupWarps;
     unsigned long long& waited = tr.waited;
-    for (int j = 0; j < nst; ++j, rg.advance(P.ns)) {
-        if (rg.slot % kGroups != group || !ok) continue;  // group g: slots g mod kGroups
-        if (!wait_full(sm, rg, P, ctl, waited)) {
-            ok = false;
-            continue;
-        }
+    auto slice = [&](const Ring& at_rg, int j, const __nv_bfloat16*& k, const __nv_bfloat16*& v) {
         const int s0 = at.a + j * P.pos_per_stage;
         const int n = min(P.pos_per_stage, at.tma_end - s0);
-        const __nv_bfloat16* st = reinterpret_cast<const __nv_bfloat16*>(sm.ring + (size_t)rg.slot * kStageBytes);
+        const __nv_bfloat16* st = reinterpret_cast<const __nv_bfloat16*>(sm.ring + (size_t)at_rg.slot * kStageBytes);
         const int p0 = n * gw / kGroupWarps, p1 = n * (gw + 1) / kGroupWarps;
-        const __nv_bfloat16* ka = st + (size_t)p0 * HD;
-        const __nv_bfloat16* va = st + (size_t)(n + p0) * HD;
-        const int na = min(8, p1 - p0), nb = p1 - p0 - na;
-        if (na > 0) pass2(ka, va, na, ka + (size_t)8 * HD, va + (size_t)8 * HD, nb, false);
-        __syncwarp();
-        if (lane == kSyncLane) mbar_arrive(smem_u32(&sm.empty[rg.slot]));
+        k = st + (size_t)p0 * HD;
+        v = st + (size_t)(n + p0) * HD;
+        return p1 - p0;
+    };
+    for (int j = 0; j < nst;) {
+        const Ring ra = rg;
+        rg.advance(P.ns);
+        const bool two = HD == 128 && j + 1 < nst;
+        const Ring rb = rg;
+        if (two) rg.advance(P.ns);
+        if (ok) {
+            if (!wait_full(sm, ra, P, ctl, waited) || (two && !wait_full(sm, rb, P, ctl, waited))) {
+                ok = false;
+            } else {
+                const __nv_bfloat16 *ka, *va, *kb, *vb;
+                int na = slice(ra, j, ka, va), nb = 0;
+                if (two) {
+                    nb = slice(rb, j + 1, kb, vb);
+                } else {  // hd 64: the stage's second block of 8
+                    nb = na > 8 ? na - 8 : 0;
+                    na -= nb;
+                    kb = ka + (size_t)8 * HD, vb = va + (size_t)8 * HD;
+                }
+                if (na == 0 && nb > 0) {  // pass2 wants a non-empty first block
+                    ka = kb, va = vb, na = nb, nb = 0;
+                }
+                if (na > 0) pass2(ka, va, na, kb, vb, nb, false);
+                __syncwarp();
+                if (lane == kSyncLane) {
+                    mbar_arrive(smem_u32(&sm.empty[ra.slot]));
+                    if (two) mbar_arrive(smem_u32(&sm.empty[rb.slot]));
+                }
+            }
+        }
+        j += two ? 2 : 1;
     }
     // the current position, appended above
     if (has_current && warp == kConsumerWarps - 1) pass2(sm.kvcur, sm.kvcur + HD, 1, sm.kvcur, sm.kvcur + HD, 0, false);
@@ -1293,7 +1322,7 @@ __global__ void __launch_bounds__(kThreads, 1) monokernel(const __grid_constant_
             if (ph == kO) {
                 load_vector(sm, reinterpret_cast<const float*>(P.arena + P.lay.o), dm.qd);
             } else if (ph == kD) {
-                load_swiglu(sm, reinterpret_cast<const float*>(P.arena + P.lay.gu), dm.F);
+                load_vector(sm, reinterpret_cast<const float*>(P.arena + P.lay.gu), dm.F);
             } else if (ph != kATT) {
                 const __nv_bfloat16* gain = reinterpret_cast<const __nv_bfloat16*>(
                     ph == kQKV ? lb + P.lay.l_attn_norm : ph == kGU ? lb + P.lay.l_ffn_norm : P.arena + P.lay.final_norm);

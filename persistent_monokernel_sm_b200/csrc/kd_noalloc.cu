@@ -71,7 +71,7 @@ extern "C" int kd_decode_noalloc(kd_ctx* ctx, const int32_t* d_tokens, int32_t n
         return at;
     };
     const size_t o_x = take((size_t)dm.d * 4), o_q = take((size_t)dm.qkv_rows * 4), o_o = take((size_t)dm.qd * 4);
-    const size_t o_hdn = take((size_t)2 * dm.F * 4);
+    const size_t o_hdn = take((size_t)dm.F * 4);
     const size_t o_part = take((size_t)v.nb * dm.r * (dm.hd + 2) * 4);
     const size_t o_ctl = take((size_t)kCtlWords * 8);
     const size_t o_tok = take((size_t)n_tokens * 4);
