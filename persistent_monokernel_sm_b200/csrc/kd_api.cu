@@ -150,11 +150,21 @@ __global__ void repack_qkv(uint8_t* dst_layer0, size_t layer_stride, size_t off,
     for (int i = threadIdx.x; i < dm.d / 8; i += blockDim.x) d[i] = s[i];
 }
 
-// dst rows (2i, 2i + 1) = (gate row i, up row i)
+// blk == 1: dst rows (2i, 2i + 1) = (gate row i, up row i). blk > 1: blocks of 2 * blk rows,
+// the gate rows of units [b * blk, (b + 1) * blk) followed by their up rows (the kernel then
+// reads a unit's gate and up rows in two consecutive stages, in the same warp).
 __global__ void repack_gu(uint8_t* dst_layer0, size_t layer_stride, size_t off, const uint16_t* wg,
-                          const uint16_t* wu, Dims dm) {
+                          const uint16_t* wu, Dims dm, int blk) {
     const int r = blockIdx.x, l = blockIdx.y;
-    const uint16_t* src = ((r & 1) ? wu : wg) + ((size_t)l * dm.F + (r >> 1)) * dm.d;
+    int unit, up;
+    if (blk == 1) {
+        unit = r >> 1, up = r & 1;
+    } else {
+        const int b = r / (2 * blk), w = r % (2 * blk);
+        up = w >= blk;
+        unit = b * blk + (up ? w - blk : w);
+    }
+    const uint16_t* src = (up ? wu : wg) + ((size_t)l * dm.F + unit) * dm.d;
     const uint4* s = reinterpret_cast<const uint4*>(src);
     uint4* d = reinterpret_cast<uint4*>(dst_layer0 + (size_t)l * layer_stride + off + (size_t)r * dm.d * 2);
     for (int i = threadIdx.x; i < dm.d / 8; i += blockDim.x) d[i] = s[i];
@@ -307,8 +317,9 @@ int kd_load_weights(kd_ctx* c, const kd_weights* w) {
     repack_qkv<<<dim3(d.qkv_rows, d.L), 128, 0, s>>>(l0, y.layer_stride, y.l_wqkv, (const uint16_t*)w->wq,
                                                       (const uint16_t*)w->wk, (const uint16_t*)w->wv, d);
     KD_CUDA(c, cudaGetLastError());
+    const int gu_rows = rows_per_stage(d.d, true);
     repack_gu<<<dim3(2 * d.F, d.L), 128, 0, s>>>(l0, y.layer_stride, y.l_wgu, (const uint16_t*)w->wg,
-                                                  (const uint16_t*)w->wu, d);
+                                                  (const uint16_t*)w->wu, d, gu_rows == kGroupWarps ? gu_rows : 1);
     KD_CUDA(c, cudaGetLastError());
     c->launches += 2;
     // RoPE table: (cos, sin) of position p times frequency theta^(-2i/hd), formed in double

@@ -150,6 +150,7 @@ struct Tracer {
 
 // Lane that performs a warp's shared-memory bookkeeping (see run_gemv).
 constexpr int kSyncLane = 31;
+static_assert(kGroupWarps == 8, "GEMV slice arithmetic assumes 8 warps per group");
 
 // ------------------------------------------------------------------ schedule geometry
 // Both the producer and the consumers enumerate the same stage sequence from these.
@@ -161,30 +162,61 @@ struct Gemv {
     int K;                // reduction length (bf16 elements per row)
     int row0, row1;       // this CTA's rows
     int R;                // rows per stage
+    int nst;              // stages
 };
 
-__device__ __forceinline__ Gemv gemv_geom(const Params& P, int phase, int l, int c) {
+// This CTA's rows of every GEMV phase, [phase][row0, row1, stages], and the residual rows
+// it owns: computed once per launch into shared memory (the 64-bit divisions that split the
+// rows over the grid would otherwise be paid by every warp at every phase).
+constexpr int kGeomOwn = 18, kGeomWords = 32;
+__device__ void cta_geometry(const Params& P, int c, int* geom) {
+    const Dims& dm = P.dm;
+    for (int phase = 0; phase < 6; ++phase) {
+        int units = 0, rpu = 1, R = 1;
+        switch (phase) {
+            case kQKV: units = dm.qkv_rows / 2; rpu = 2; R = P.rows_qkv; break;
+            case kO: units = dm.d; R = P.rows_o; break;
+            case kGU:  // blocks of R gate rows then R up rows when a warp owns a row, else pairs
+                R = P.rows_gu;
+                if (R == kGroupWarps) units = dm.F / R, rpu = 2 * R;
+                else units = dm.F, rpu = 2;
+                break;
+            case kD: units = dm.d; R = P.rows_d; break;
+            case kLM: units = dm.V; R = P.rows_lm; break;
+            default: break;
+        }
+        const int row0 = (int)((long long)units * c / P.nb) * rpu;
+        const int row1 = (int)((long long)units * (c + 1) / P.nb) * rpu;
+        geom[3 * phase] = row0;
+        geom[3 * phase + 1] = row1;
+        geom[3 * phase + 2] = (row1 - row0 + R - 1) / R;
+    }
+    geom[kGeomOwn] = (int)((long long)dm.d * c / P.nb);
+    geom[kGeomOwn + 1] = (int)((long long)dm.d * (c + 1) / P.nb);
+}
+
+__device__ __forceinline__ Gemv gemv_geom(const Params& P, const int* geom, int phase, int l) {
     const Dims& dm = P.dm;
     const uint8_t* lb = P.arena + P.lay.layer0 + (size_t)l * P.lay.layer_stride;
     Gemv g;
-    int units, rpu;
     switch (phase) {
-        case kQKV: g.base = lb + P.lay.l_wqkv; g.K = dm.d; units = dm.qkv_rows / 2; rpu = 2; g.R = P.rows_qkv; break;
-        case kO: g.base = lb + P.lay.l_wo; g.K = dm.qd; units = dm.d; rpu = 1; g.R = P.rows_o; break;
-        case kGU: g.base = lb + P.lay.l_wgu; g.K = dm.d; units = dm.F; rpu = 2; g.R = P.rows_gu; break;
-        case kD: g.base = lb + P.lay.l_wd; g.K = dm.F; units = dm.d; rpu = 1; g.R = P.rows_d; break;
-        default: g.base = P.arena + P.lay.lm_head; g.K = dm.d; units = dm.V; rpu = 1; g.R = P.rows_lm; break;
+        case kQKV: g.base = lb + P.lay.l_wqkv; g.K = dm.d; g.R = P.rows_qkv; break;
+        case kO: g.base = lb + P.lay.l_wo; g.K = dm.qd; g.R = P.rows_o; break;
+        case kGU: g.base = lb + P.lay.l_wgu; g.K = dm.d; g.R = P.rows_gu; break;
+        case kD: g.base = lb + P.lay.l_wd; g.K = dm.F; g.R = P.rows_d; break;
+        default: g.base = P.arena + P.lay.lm_head; g.K = dm.d; g.R = P.rows_lm; break;
     }
-    g.row0 = (int)((long long)units * c / P.nb) * rpu;
-    g.row1 = (int)((long long)units * (c + 1) / P.nb) * rpu;
+    g.row0 = geom[3 * phase];
+    g.row1 = geom[3 * phase + 1];
+    g.nst = geom[3 * phase + 2];
     return g;
 }
-__device__ __forceinline__ int gemv_stages(const Gemv& g) { return (g.row1 - g.row0 + g.R - 1) / g.R; }
 
 struct Attn {
     int g, piece;  // kv head, piece index (g < 0: this CTA has no piece)
     int a, b;      // positions [a, b) of the piece (b may include the current position)
     int tma_end;   // [a, tma_end) streamed through the ring; position p handled directly
+    int nst;       // ring stages of the piece
 };
 
 __device__ __forceinline__ Attn attn_geom(const Params& P, int p, int c) {
@@ -193,7 +225,7 @@ __device__ __forceinline__ Attn attn_geom(const Params& P, int p, int c) {
     if (c >= A * P.dm.Hkv) {
         at.g = -1;
         at.piece = 0;
-        at.a = at.b = at.tma_end = 0;
+        at.a = at.b = at.tma_end = at.nst = 0;
         return at;
     }
     at.g = c / A;
@@ -203,10 +235,8 @@ __device__ __forceinline__ Attn attn_geom(const Params& P, int p, int c) {
     at.b = (int)(T * (at.piece + 1) / A);
     at.tma_end = at.b < p ? at.b : p;
     if (at.tma_end < at.a) at.tma_end = at.a;
+    at.nst = (at.tma_end - at.a + P.pos_per_stage - 1) / P.pos_per_stage;
     return at;
-}
-__device__ __forceinline__ int attn_stages(const Params& P, const Attn& at) {
-    return (at.tma_end - at.a + P.pos_per_stage - 1) / P.pos_per_stage;
 }
 
 // The LM head runs at steps that pick a token, or at every step when logits are dumped.
@@ -235,12 +265,14 @@ struct Smem {
     int* scnt;              // per-stage arrival counts [slot]
     float* xown;            // the residual rows this CTA owns (updated by O and D)
     __nv_bfloat16* kvcur;   // the current position's K and V row of the head being attended
+    int* geom;              // this CTA's GEMV rows per phase and owned residual rows (cta_geometry)
+    Attn* att;              // this step's attention piece (consumers)
 };
 
 // Byte offsets of the shared-memory regions; each starts on a 128-byte boundary (vector
 // loads and bulk-copy destinations need 16). Used by the kernel and for the launch size.
 struct SmemLayout {
-    size_t ring, xs, qs, rope, red, best, flag, full, empty, sp, scnt, xown, kvcur, total;
+    size_t ring, xs, qs, rope, red, best, flag, full, empty, sp, scnt, xown, kvcur, geom, att, total;
 };
 __host__ __device__ inline SmemLayout smem_layout(int ns, int xs_floats, int xown_floats) {
     SmemLayout L;
@@ -263,6 +295,8 @@ __host__ __device__ inline SmemLayout smem_layout(int ns, int xs_floats, int xow
     L.scnt = take((size_t)kMaxStages * 4);
     L.xown = take((size_t)xown_floats * 4);
     L.kvcur = take(2 * 128 * 2);
+    L.geom = take((size_t)kGeomWords * 4);
+    L.att = take(sizeof(Attn));
     L.total = off;
     return L;
 }
@@ -283,6 +317,8 @@ __device__ __forceinline__ Smem carve(const Params& P, uint8_t* base) {
     s.scnt = reinterpret_cast<int*>(base + L.scnt);
     s.xown = reinterpret_cast<float*>(base + L.xown);
     s.kvcur = reinterpret_cast<__nv_bfloat16*>(base + L.kvcur);
+    s.geom = reinterpret_cast<int*>(base + L.geom);
+    s.att = reinterpret_cast<Attn*>(base + L.att);
     return s;
 }
 
@@ -466,7 +502,7 @@ struct StepCtx {
 // Output of one finished GEMV row (global row index `row`, value y): stored raw for the
 // Q/K/V projections (RoPE and the KV-cache append are applied where they are consumed),
 // the FFN hidden value silu(gate) * up for a gate/up pair (y is already that value; `row` is
-// the pair's gate row), added into the residual for O and down (the CTA owns those rows and
+// the pair's index), added into the residual for O and down (the CTA owns those rows and
 // keeps them in shared memory, so no read-back from L2), and for the LM head dumped when
 // requested and folded into this thread's running argmax.
 __device__ __forceinline__ void row_out(const Params& P, const Smem& sm, int phase, int row, float y, StepCtx& sc,
@@ -475,7 +511,7 @@ __device__ __forceinline__ void row_out(const Params& P, const Smem& sm, int pha
     if (phase == kQKV) {
         __stcg(reinterpret_cast<float*>(arena + P.lay.qkv) + row, y);
     } else if (phase == kGU) {
-        __stcg(reinterpret_cast<float*>(arena + P.lay.gu) + (row >> 1), y);  // hidden value of pair row / 2
+        __stcg(reinterpret_cast<float*>(arena + P.lay.gu) + row, y);  // `row`: the pair (hidden unit) index
     } else if (phase == kO || phase == kD) {
         const float v = sm.xown[row - own0] + y;
         sm.xown[row - own0] = v;
@@ -509,17 +545,18 @@ __device__ __forceinline__ void run_gemv_t(const Params& P, const Smem& sm_ref, 
     Ring rg = rg_ref;
     StepCtx sc = sc_ref;
     bool ok = ok_ref;
-    const Gemv g = gemv_geom(P, phase, l, blockIdx.x);
-    const int nst = gemv_stages(g);
+    const Gemv g = gemv_geom(P, sm.geom, phase, l);
+    const int nst = g.nst;
     const int ns = P.ns;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int group = warp / kGroupWarps, gw = warp % kGroupWarps;
-    const int KS = kGroupWarps / g.R;  // slices per row (rows_per_stage gives R in {1, 2, 4, 8})
-    const int row = gw / KS, ks = gw % KS;
+    // slices per row: rows_per_stage gives R in {1, 2, 4, 8}, so KS is a power of two too
+    const int lks = 3 - (__ffs(g.R) - 1), KS = 1 << lks;
+    const int row = gw >> lks, ks = gw & (KS - 1);
     const int nch = g.K >> 3;
-    const int c0 = nch * ks / KS, c1 = nch * (ks + 1) / KS;  // at most 32 * kMaxChunks chunks
+    const int c0 = (nch * ks) >> lks, c1 = (nch * (ks + 1)) >> lks;  // at most 32 * kMaxChunks chunks
     const size_t rowb = (size_t)g.K * 2;
-    const int own0 = (int)((long long)P.dm.d * blockIdx.x / P.nb);
+    const int own0 = sm.geom[kGeomOwn];
     unsigned long long& waited = tr.waited;
 
     // this lane's activation chunks: c = c0 + lane + 32 i
@@ -560,7 +597,7 @@ __device__ __forceinline__ void run_gemv_t(const Params& P, const Smem& sm_ref, 
     };
     // per-stage completion: release the slot and put the row(s) out
     auto finish = [&](const Ring& at_rg, int r0, int n, float part) {
-        if (KS == 1 && phase != kGU) {  // this warp owns the whole row
+        if (KS == 1) {  // this warp owns the whole row
             __syncwarp();
             if (lane == kSyncLane) mbar_arrive(smem_u32(&sm.empty[at_rg.slot]));  // done with the stage
             if (lane == 0 && row < n) row_out(P, sm, phase, r0 + row, part, sc, own0);
@@ -589,7 +626,8 @@ __device__ __forceinline__ void run_gemv_t(const Params& P, const Smem& sm_ref, 
             // rows come in (gate, up) pairs, lane 2j holding gate j and lane 2j + 1 up j:
             // the FFN hidden value silu(gate) * up is formed here, once, for the D phase
             const float up = __shfl_down_sync(0xffffffffu, tot, 1);
-            if (lane < n && (lane & 1) == 0) row_out(P, sm, phase, r0 + lane, tot / (1.0f + expf(-tot)) * up, sc, own0);
+            if (lane < n && (lane & 1) == 0)
+                row_out(P, sm, phase, (r0 + lane) >> 1, tot / (1.0f + expf(-tot)) * up, sc, own0);
         } else if (lane < n) {
             row_out(P, sm, phase, r0 + lane, tot, sc, own0);
         }
@@ -634,6 +672,17 @@ __device__ __forceinline__ void run_gemv_t(const Params& P, const Smem& sm_ref, 
             pa += __shfl_xor_sync(0xffffffffu, pa, o);
             pb += __shfl_xor_sync(0xffffffffu, pb, o);
         }
+        if (phase == kGU && KS == 1) {
+            // block layout: stage a holds R gate rows, stage b the R up rows of the same units,
+            // so this warp has both halves of its unit and forms silu(gate) * up itself
+            __syncwarp();
+            if (lane == kSyncLane) {
+                mbar_arrive(smem_u32(&sm.empty[ra.slot]));
+                mbar_arrive(smem_u32(&sm.empty[rb.slot]));
+            }
+            if (lane == 0 && row < na) row_out(P, sm, phase, (ra0 >> 1) + row, pa / (1.0f + expf(-pa)) * pb, sc, own0);
+            continue;
+        }
         finish(ra, ra0, na, pa);
         if (two) finish(rb, rb0, nb, pb);
     }
@@ -654,13 +703,14 @@ __device__ __forceinline__ void run_gemv_t(const Params& P, const Smem& sm_ref, 
 
 // Chunks (8 elements) per lane of every warp's slice when that count is exact, else 0.
 __device__ __forceinline__ int gemv_exact_chunks(int K, int R) {
-    const int KS = kGroupWarps / R, nch = K >> 3;
-    return nch % (32 * KS) == 0 && nch / (32 * KS) <= kMaxChunks ? nch / (32 * KS) : 0;
+    const int lks = 3 - (__ffs(R) - 1);  // log2(kGroupWarps / R)
+    const int nch = K >> 3, per = nch >> (5 + lks);
+    return (per << (5 + lks)) == nch && per <= kMaxChunks ? per : 0;
 }
 
 __device__ __forceinline__ void run_gemv(const Params& P, const Smem& sm, unsigned long long* ctl, int phase, int l,
                                       Ring& rg, StepCtx& sc, bool& ok, Tracer& tr) {
-    const Gemv g = gemv_geom(P, phase, l, blockIdx.x);
+    const Gemv g = gemv_geom(P, sm.geom, phase, l);
     switch (gemv_exact_chunks(g.K, g.R)) {
         case 1: run_gemv_t<1>(P, sm, ctl, phase, l, rg, sc, ok, tr); break;
         case 2: run_gemv_t<2>(P, sm, ctl, phase, l, rg, sc, ok, tr); break;
@@ -709,7 +759,7 @@ __device__ __forceinline__ void run_attention(const Params& P, const Smem& sm_re
     const Dims& dm = P.dm;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
     const int pj = lane >> 2, qq = lane & 3;
-    const Attn at = attn_geom(P, sc.p, blockIdx.x);
+    const Attn at = *sm.att;  // this step's piece, set at the step start
     if (at.g < 0) return;  // uniform across the CTA
     const int r = dm.r, A = P.attn_pieces;
     const float qscale = 1.4426950408889634f / sqrtf((float)HD);  // log2(e) / sqrt(hd)
@@ -857,7 +907,7 @@ __device__ __forceinline__ void run_attention(const Params& P, const Smem& sm_re
     // hd 128, at most 16 (the two blocks of one pass) with hd 64. With hd 128 a warp takes two
     // stages per pass, one block from each, so each online-softmax update covers 16 positions.
     static_assert(kGroups == 1, "attention stages assume one consumer group");
-    const int nst = attn_stages(P, at);
+    const int nst = at.nst;
     const int gw = warp % kGroupWarps;
     unsigned long long& waited = tr.waited;
     auto slice = [&](const Ring& at_rg, int j, const __nv_bfloat16*& k, const __nv_bfloat16*& v) {
@@ -1000,6 +1050,8 @@ __device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes
 struct Cursor {
     int t = 0, l = 0, ph = 0, j = 0, nst = 0;
     bool done = false;
+    const int* geom = nullptr;  // cta_geometry
+    int at_t = -1;              // step whose attention piece `at` holds
     Gemv g;
     Attn at;
 
@@ -1011,11 +1063,14 @@ struct Cursor {
     __device__ void enter(const Params& P) {
         j = 0;
         if (ph == kATT) {
-            at = attn_geom(P, P.pos0 + t, blockIdx.x);
-            nst = at.g < 0 ? 0 : attn_stages(P, at);
+            if (at_t != t) {  // once per step: the piece only moves with the position
+                at = attn_geom(P, P.pos0 + t, blockIdx.x);
+                at_t = t;
+            }
+            nst = at.g < 0 ? 0 : at.nst;
         } else {
-            g = gemv_geom(P, ph, ph == kLM ? 0 : l, blockIdx.x);
-            nst = gemv_stages(g);
+            g = gemv_geom(P, geom, ph, ph == kLM ? 0 : l);
+            nst = g.nst;
         }
     }
     __device__ void settle(const Params& P) {
@@ -1185,6 +1240,7 @@ struct Producer {
         const long long c_start = clock64();
         bool ok = true;
         Cursor ld, pf;
+        ld.geom = pf.geom = sm.geom;
         ld.begin(P);
         pf.begin(P);
         for (int i = 0; i < P.prefetch && !pf.done; ++i, pf.next(P)) prefetch(pf);
@@ -1236,6 +1292,7 @@ __global__ void __launch_bounds__(kThreads, 1) monokernel(const __grid_constant_
             sm.scnt[s] = 0;
         }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        cta_geometry(P, blockIdx.x, sm.geom);
         // Barrier count at launch: a multiple of nb plus arrivals of CTAs that already
         // reached this launch's first barrier (which cannot complete before we arrive).
         const uint64_t raw = ld_acquire_u64(ctl + kCtlBar);
@@ -1270,8 +1327,7 @@ __global__ void __launch_bounds__(kThreads, 1) monokernel(const __grid_constant_
         tr.rows = P.trace_rows;
         tr.mark(0);
     }
-    const int own0 = (int)((long long)dm.d * blockIdx.x / P.nb);
-    const int own1 = (int)((long long)dm.d * (blockIdx.x + 1) / P.nb);
+    const int own0 = sm.geom[kGeomOwn], own1 = sm.geom[kGeomOwn + 1];
 
     for (int t = 0; t < P.steps && ok; ++t) {
         sc.t = t;
@@ -1294,6 +1350,7 @@ __global__ void __launch_bounds__(kThreads, 1) monokernel(const __grid_constant_
             }
             sm.flag[2] = tok;
         }
+        if (tid == 32) *sm.att = attn_geom(P, sc.p, blockIdx.x);  // this step's attention piece
         if (tid < dm.hd / 2)  // this position's RoPE row (cos, sin per pair)
             sm.rope[tid] = __ldg(reinterpret_cast<const float2*>(P.arena + P.lay.rope) + (size_t)sc.p * (dm.hd / 2) + tid);
         consumer_sync();
