@@ -75,10 +75,10 @@ Layout make_layout(const Dims& d) {
     y.kcache = take(kv);
     y.vcache = take(kv);
     y.kv_bytes = 2 * kv;
-    y.x = take(D * 4);
-    y.qkv = take((size_t)d.qkv_rows * 4);  // raw q/k/v projections (repacked row order)
-    y.o = take((size_t)d.qd * 4);
-    y.gu = take((size_t)d.F * 4);  // FFN hidden vector silu(gate) * up
+    y.x = take(2 * D * 8);                 // tagged: residual after O, after D
+    y.qkv = take((size_t)d.qkv_rows * 8);  // tagged raw q/k/v projections (repacked row order)
+    y.o = take((size_t)d.qd * 8);          // tagged attention output
+    y.gu = take((size_t)d.F * 8);          // tagged FFN hidden vector silu(gate) * up
     y.part = take((size_t)kMaxGrid * d.r * (d.hd + 2) * 4);
     y.ctl = take((size_t)kCtlWords * 8);
     y.tokens_in = take((size_t)d.S * 4);
@@ -102,6 +102,7 @@ struct kd_ctx {
     long long launches;
     long long timeout_ns;
     int prefetch, inflight;
+    uint32_t tag;  // tag base of the next launch (advanced by the phases each launch runs)
     unsigned long long* trace;
     int trace_every, trace_rows;
     char err[512];
@@ -258,7 +259,18 @@ int kd_create(const kd_config* cfg, void* d_arena, size_t arena_bytes, void* str
         if (d.F > xs) xs = d.F;
         const int merge = kConsumerWarps * d.r * (d.hd + 2);
         if (merge > xs) xs = merge;
-        if (kMaxGroup * c->pieces + kMaxGroup > xs) xs = kMaxGroup * c->pieces + kMaxGroup;  // combine weights
+        // GEMV phases whose rows are split over several warps keep [row][slice] sums in xs
+        {
+            const int K[5] = {d.d, d.qd, d.d, d.F, d.d};
+            const long long units[5] = {d.qkv_rows / 2, d.d, d.F, d.d, d.V};
+            const int rpu[5] = {2, 1, 2, 1, 1};
+            for (int i = 0; i < 5; ++i) {
+                const int R = rows_per_stage(K[i], false);
+                if (R >= kGroupWarps) continue;
+                const long long rows = (units[i] + c->nb - 1) / c->nb * rpu[i];
+                if (rows * (kGroupWarps / R) > xs) xs = (int)(rows * (kGroupWarps / R));
+            }
+        }
         c->xs_floats = (xs + 31) & ~31;
         c->xown_floats = (d.d + c->nb - 1) / c->nb + 1;
         Params p{};
@@ -281,7 +293,10 @@ int kd_create(const kd_config* cfg, void* d_arena, size_t arena_bytes, void* str
         }
     }
     if (rc == KD_OK) {
+        // control words and the tagged activation buffers start at zero: tag 0 is never
+        // expected (the first launch's phases carry tags 1, 2, ...)
         cudaError_t e = cudaMemsetAsync(c->arena + c->lay.ctl, 0, (size_t)kCtlWords * 8, c->stream);
+        if (e == cudaSuccess) e = cudaMemsetAsync(c->arena + c->lay.x, 0, c->lay.part - c->lay.x, c->stream);
         if (e != cudaSuccess) rc = fail(c, KD_ECUDA, "cudaMemsetAsync: %s", cudaGetErrorString(e));
     }
     if (rc != KD_OK) {
@@ -417,6 +432,7 @@ int kd_decode(kd_ctx* c, int32_t n_gen, int32_t* d_tokens_out, float* d_logits_o
     p.timeout_ns = c->timeout_ns;
     p.prefetch = c->prefetch;
     p.inflight = c->inflight;
+    p.tag0 = c->tag;
     p.trace = c->trace;
     p.trace_every = c->trace_every;
     p.trace_rows = c->trace_rows;
@@ -424,6 +440,7 @@ int kd_decode(kd_ctx* c, int32_t n_gen, int32_t* d_tokens_out, float* d_logits_o
     launch_decode(p, c->stream, c->smem, &e);
     if (e != 0) return fail(c, KD_ECUDA, "cooperative launch failed: %s", cudaGetErrorString((cudaError_t)e));
     c->launches += 1;
+    c->tag += (uint32_t)launch_phases(c->dm, steps, c->n_pending, d_logits_out != nullptr);
     c->pos += steps;
     c->n_pending = 1;
     return KD_OK;

@@ -99,6 +99,24 @@ __device__ __forceinline__ unsigned int atom_add_acq_rel_u32(unsigned int* p, un
     asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
     return old;
 }
+
+// Tagged activation words: value (fp32 bits) in the low half, the producing phase's tag in
+// the high half. A 64-bit store is single-copy atomic, so a reader that sees the tag sees
+// the value written with it; no fence or barrier orders the two.
+__device__ __forceinline__ void st_tagged(unsigned long long* p, float v, uint32_t tag) {
+    const unsigned long long w = ((unsigned long long)tag << 32) | (unsigned long long)__float_as_uint(v);
+    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(w) : "memory");
+}
+// Two consecutive tagged words (16-byte aligned); each 8-byte element is read atomically.
+__device__ __forceinline__ ulonglong2 ld_tagged2(const unsigned long long* p) {
+    ulonglong2 w;
+    asm volatile("ld.relaxed.gpu.global.v2.u64 {%0, %1}, [%2];" : "=l"(w.x), "=l"(w.y) : "l"(p));
+    return w;
+}
+__device__ __forceinline__ float tagged_value(unsigned long long w) { return __uint_as_float((uint32_t)w); }
+__device__ __forceinline__ bool tagged_pair_is(const ulonglong2& w, uint32_t tag) {
+    return (uint32_t)(w.x >> 32) == tag && (uint32_t)(w.y >> 32) == tag;
+}
 __device__ __forceinline__ void consumer_sync() {
     asm volatile("bar.sync 1, %0;" ::"n"(kConsumerThreads) : "memory");
 }
@@ -128,7 +146,7 @@ __device__ __forceinline__ void raise_timeout(unsigned long long* ctl, int where
 }
 
 // Where a wait gave up or an input was refused: (what << 24) | (cta << 8) | detail.
-enum { kWhereFull = 1, kWhereEmpty = 2, kWhereGrid = 3, kWhereKv = 4, kWhereToken = 5 };
+enum { kWhereFull = 1, kWhereEmpty = 2, kWhereGrid = 3, kWhereKv = 4, kWhereToken = 5, kWhereData = 6 };
 __device__ __forceinline__ int where_code(int what, int detail) {
     return (what << 24) | ((int)blockIdx.x << 8) | (detail & 0xff);
 }
@@ -243,10 +261,16 @@ __device__ __forceinline__ Attn attn_geom(const Params& P, int p, int c) {
 __device__ __forceinline__ bool step_has_head(const Params& P, int t) {
     return P.dump || t >= P.n_pending - 1;
 }
-// Grid barriers completed before step s begins.
-__device__ __forceinline__ long long barriers_before_step(const Params& P, int s) {
+// Phases run before step s begins (5 per layer, plus the LM head at steps that have one).
+__device__ __forceinline__ long long phases_before_step(const Params& P, int s) {
     long long heads = P.dump ? s : (s - (P.n_pending - 1) > 0 ? s - (P.n_pending - 1) : 0);
     return (long long)s * 5 * P.dm.L + heads;
+}
+// Tag of phase q of step t (q = 5 * layer + phase, or 5 * L for the LM head). Every
+// activation element a phase writes for other CTAs carries its tag in the same 64-bit word
+// as the value, so a reader polls the data itself instead of a grid barrier.
+__device__ __forceinline__ uint32_t phase_tag(const Params& P, int t, int q) {
+    return P.tag0 + 1u + (uint32_t)(phases_before_step(P, t) + q);
 }
 
 // ------------------------------------------------------------------ shared memory
@@ -275,7 +299,7 @@ struct SmemLayout {
     size_t ring, xs, qs, rope, red, best, flag, full, empty, sp, scnt, xown, kvcur, geom, att, total;
 };
 __host__ __device__ inline SmemLayout smem_layout(int ns, int xs_floats, int xown_floats) {
-    SmemLayout L;
+    SmemLayout L{};
     size_t off = 0;
     auto take = [&](size_t bytes) {
         const size_t at = off;
@@ -382,6 +406,46 @@ __device__ __forceinline__ bool wait_full(const Smem& sm, const Ring& rg, const 
     }
 }
 
+// End of a phase inside a step: every consumer warp is done with xs, and the CTA agrees on
+// whether every wait succeeded (a failed CTA stops; the others stop at their next wait, which
+// sees the status word).
+__device__ __forceinline__ bool phase_end(bool local_ok, Tracer& tr) {
+    const bool cta_ok = consumer_sync_and(local_ok);
+    if (threadIdx.x == 0) {
+        tr.mark(2);
+        tr.mark(3);
+        tr.next();
+        tr.mark(0);
+    }
+    return cta_ok;
+}
+
+// Re-read a 16-byte pair of tagged words until both carry `tag` (the first read was issued
+// by the caller together with its other loads). Gives up, with the device status set, when
+// another wait has failed or after the time limit; `what` identifies the buffer.
+// Returns the pair; its tags differ from `tag` only when the wait gave up.
+__device__ __noinline__ ulonglong2 poll_pair(const unsigned long long* p, uint32_t tag, const Params& P,
+                                             unsigned long long* ctl, int what) {
+    const uint64_t t0 = globaltimer();
+    for (uint32_t it = 1;; ++it) {
+        const ulonglong2 w = ld_tagged2(p);
+        if (tagged_pair_is(w, tag)) return w;
+        if ((it & 31) == 0) {
+            if (read_status(ctl) != 0) return w;
+            if (globaltimer() - t0 > (uint64_t)P.timeout_ns) {
+                raise_timeout(ctl, where_code(kWhereData, what));
+                return w;
+            }
+        }
+    }
+}
+__device__ __forceinline__ bool get_pair(const unsigned long long* p, uint32_t tag, ulonglong2& w, const Params& P,
+                                         unsigned long long* ctl, int what) {
+    if (tagged_pair_is(w, tag)) return true;
+    w = poll_pair(p, tag, P, ctl, what);
+    return tagged_pair_is(w, tag);
+}
+
 // Grid-wide barrier among the consumer warps of all CTAs. `epoch` counts barriers this
 // launch has completed; arrivals accumulate in one monotonic counter, so there is no
 // reset race and a barrier completes when the counter reaches base + epoch * nb.
@@ -436,23 +500,57 @@ __device__ __forceinline__ void sts128(float* p, float4 v) {
     asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(smem_u32(p)), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w));
 }
 
-// xs <- x * rsqrt(mean(x^2) + eps) * g in split layout. src_f32 (global, written during
-// the launch) or src_bf16 (an embedding row, read-only).
-__device__ __forceinline__ void load_rmsnorm(const Smem& sm, const float* src_f32, const __nv_bfloat16* src_bf16,
-                             const __nv_bfloat16* gain, int K, float eps) {
+// Tagged vectors are read two float4 groups (four 16-byte loads) per thread at a time, all
+// four loads issued before any tag is checked, so a pair of groups whose data is ready costs
+// one L2 round trip; a stale pair is re-polled until it carries `tag` (`ok` turns false if
+// that wait gives up). The loads go to named registers: arrays written by asm get a stack
+// slot.
+struct Tagged2x4 {
+    ulonglong2 a0, b0, a1, b1;
+};
+__device__ __forceinline__ void load_groups(const unsigned long long* src, int k0, int k1, bool h1, Tagged2x4& t) {
+    t.a0 = ld_tagged2(src + k0);
+    t.b0 = ld_tagged2(src + k0 + 2);
+    if (h1) {
+        t.a1 = ld_tagged2(src + k1);
+        t.b1 = ld_tagged2(src + k1 + 2);
+    }
+}
+__device__ __forceinline__ float4 group_value(const unsigned long long* src, int k, uint32_t tag, ulonglong2 a, ulonglong2 b,
+                                              const Params& P, unsigned long long* ctl, int what, bool& ok) {
+    if (!get_pair(src + k, tag, a, P, ctl, what) || !get_pair(src + k + 2, tag, b, P, ctl, what)) ok = false;
+    return make_float4(tagged_value(a.x), tagged_value(a.y), tagged_value(b.x), tagged_value(b.y));
+}
+
+// xs <- x * rsqrt(mean(x^2) + eps) * g in split layout. src_ll: a tagged vector written
+// during the launch by the phase with tag `tag`; else src_bf16, an embedding row.
+__device__ __forceinline__ void load_rmsnorm(const Smem& sm, const unsigned long long* src_ll, uint32_t tag,
+                                             const __nv_bfloat16* src_bf16, const __nv_bfloat16* gain, int K, float eps,
+                                             const Params& P, unsigned long long* ctl, bool& ok) {
     const int tid = threadIdx.x;
+    constexpr int step = kConsumerThreads * 4;
     float ss = 0.f;
-#pragma unroll 4
-    for (int k = tid * 4; k < K; k += kConsumerThreads * 4) {
-        float4 v;
-        if (src_f32) {
-            v = __ldcg(reinterpret_cast<const float4*>(src_f32 + k));
+    for (int k0 = tid * 4; k0 < K; k0 += 2 * step) {
+        const int k1 = k0 + step;
+        const bool h1 = k1 < K;
+        float4 v0, v1;
+        if (src_ll) {
+            Tagged2x4 t;
+            load_groups(src_ll, k0, k1, h1, t);
+            v0 = group_value(src_ll, k0, tag, t.a0, t.b0, P, ctl, 1, ok);
+            if (h1) v1 = group_value(src_ll, k1, tag, t.a1, t.b1, P, ctl, 1, ok);
         } else {
-            const uint2 w = __ldg(reinterpret_cast<const uint2*>(src_bf16 + k));
-            v = make_float4(bf_lo(w.x), bf_hi(w.x), bf_lo(w.y), bf_hi(w.y));
+            const uint2 e0 = __ldg(reinterpret_cast<const uint2*>(src_bf16 + k0));
+            const uint2 e1 = h1 ? __ldg(reinterpret_cast<const uint2*>(src_bf16 + k1)) : make_uint2(0, 0);
+            v0 = make_float4(bf_lo(e0.x), bf_hi(e0.x), bf_lo(e0.y), bf_hi(e0.y));
+            v1 = make_float4(bf_lo(e1.x), bf_hi(e1.x), bf_lo(e1.y), bf_hi(e1.y));
         }
-        ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
-        sts128(&sm.xs[xs_index(k, K)], v);
+        ss += v0.x * v0.x + v0.y * v0.y + v0.z * v0.z + v0.w * v0.w;
+        sts128(&sm.xs[xs_index(k0, K)], v0);
+        if (h1) {
+            ss += v1.x * v1.x + v1.y * v1.y + v1.z * v1.z + v1.w * v1.w;
+            sts128(&sm.xs[xs_index(k1, K)], v1);
+        }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
@@ -475,11 +573,18 @@ __device__ __forceinline__ void load_rmsnorm(const Smem& sm, const float* src_f3
     consumer_sync();
 }
 
-// xs <- src (fp32, written during the launch).
-__device__ __forceinline__ void load_vector(const Smem& sm, const float* src, int K) {
-#pragma unroll 4
-    for (int k = threadIdx.x * 4; k < K; k += kConsumerThreads * 4)
-        sts128(&sm.xs[xs_index(k, K)], __ldcg(reinterpret_cast<const float4*>(src + k)));
+// xs <- a tagged vector written during the launch by the phase with tag `tag`.
+__device__ __forceinline__ void load_vector(const Smem& sm, const unsigned long long* src, uint32_t tag, int K,
+                                            const Params& P, unsigned long long* ctl, bool& ok) {
+    constexpr int step = kConsumerThreads * 4;
+    for (int k0 = threadIdx.x * 4; k0 < K; k0 += 2 * step) {
+        const int k1 = k0 + step;
+        const bool h1 = k1 < K;
+        Tagged2x4 t;
+        load_groups(src, k0, k1, h1, t);
+        sts128(&sm.xs[xs_index(k0, K)], group_value(src, k0, tag, t.a0, t.b0, P, ctl, 2, ok));
+        if (h1) sts128(&sm.xs[xs_index(k1, K)], group_value(src, k1, tag, t.a1, t.b1, P, ctl, 2, ok));
+    }
     consumer_sync();
 }
 
@@ -496,26 +601,28 @@ __device__ __forceinline__ int key_index(unsigned long long key) {
 
 struct StepCtx {
     int t, p, l;
+    uint32_t tag;                // tag of the phase being run (its outputs carry it)
     unsigned long long lm_best;  // running argmax key of this warp (lane 0)
 };
 
-// Output of one finished GEMV row (global row index `row`, value y): stored raw for the
-// Q/K/V projections (RoPE and the KV-cache append are applied where they are consumed),
-// the FFN hidden value silu(gate) * up for a gate/up pair (y is already that value; `row` is
-// the pair's index), added into the residual for O and down (the CTA owns those rows and
-// keeps them in shared memory, so no read-back from L2), and for the LM head dumped when
-// requested and folded into this thread's running argmax.
+// Output of one finished GEMV row (global row index `row`, value y), tagged with the phase:
+// stored raw for the Q/K/V projections (RoPE and the KV-cache append are applied where
+// they are consumed), the FFN hidden value silu(gate) * up for a gate/up pair (y is already
+// that value; `row` is the pair's index), added into the residual for O and down (the CTA
+// owns those rows and keeps them in shared memory, so no read-back from L2; O's results go
+// to x copy 0, D's to copy 1), and for the LM head dumped when requested and folded into
+// this thread's running argmax.
 __device__ __forceinline__ void row_out(const Params& P, const Smem& sm, int phase, int row, float y, StepCtx& sc,
                                         int own0) {
-    uint8_t* arena = const_cast<uint8_t*>(P.arena);
+    unsigned long long* arena = reinterpret_cast<unsigned long long*>(const_cast<uint8_t*>(P.arena));
     if (phase == kQKV) {
-        __stcg(reinterpret_cast<float*>(arena + P.lay.qkv) + row, y);
+        st_tagged(arena + P.lay.qkv / 8 + row, y, sc.tag);
     } else if (phase == kGU) {
-        __stcg(reinterpret_cast<float*>(arena + P.lay.gu) + row, y);  // `row`: the pair (hidden unit) index
+        st_tagged(arena + P.lay.gu / 8 + row, y, sc.tag);  // `row`: the pair (hidden unit) index
     } else if (phase == kO || phase == kD) {
         const float v = sm.xown[row - own0] + y;
         sm.xown[row - own0] = v;
-        __stcg(reinterpret_cast<float*>(arena + P.lay.x) + row, v);
+        st_tagged(arena + P.lay.x / 8 + (phase == kO ? 0 : P.dm.d) + row, v, sc.tag);
     } else {
         if (P.dump) __stcg(P.logits_out + (size_t)sc.t * P.dm.V + row, y);
         const unsigned long long key = argmax_key(y, row);
@@ -573,6 +680,12 @@ __device__ __forceinline__ void run_gemv_t(const Params& P, const Smem& sm_ref, 
         xr[i][0] = a.x, xr[i][1] = a.y, xr[i][2] = a.z, xr[i][3] = a.w;
         xr[i][4] = b.x, xr[i][5] = b.y, xr[i][6] = b.z, xr[i][7] = b.w;
     }
+    if (threadIdx.x == 0) tr.mark(7);  // activation slice in registers
+    // When rows are split over KS > 1 warps, each warp's slice sums go to xs (free once every
+    // warp holds its activation slice) as [local row][slice] and are added up, in slice order,
+    // when the phase's stages are done: no per-stage cross-warp handshake.
+    float* pp = sm.xs;
+    if (KS > 1) consumer_sync();
 
     // Stages are taken two at a time (this group's next two): their 16 chunk loads and the
     // two cross-lane reductions interleave, and the per-stage bookkeeping is paid once per pair.
@@ -595,41 +708,13 @@ __device__ __forceinline__ void run_gemv_t(const Params& P, const Smem& sm_ref, 
         }
         s = (a0 + a1) + (a2 + a3);
     };
-    // per-stage completion: release the slot and put the row(s) out
-    auto finish = [&](const Ring& at_rg, int r0, int n, float part) {
-        if (KS == 1) {  // this warp owns the whole row
-            __syncwarp();
-            if (lane == kSyncLane) mbar_arrive(smem_u32(&sm.empty[at_rg.slot]));  // done with the stage
-            if (lane == 0 && row < n) row_out(P, sm, phase, r0 + row, part, sc, own0);
-            return;
-        }
-        float* sp = sm.sp + (size_t)at_rg.slot * kMaxRows;  // [row * KS + slice]: R * KS = 8 values
-        int last = 0;
-        if (lane == kSyncLane) {
-            if (row < n) sp[row * KS + ks] = part;
-            __threadfence_block();
-            last = atomicAdd(&sm.scnt[at_rg.slot], 1) == kGroupWarps - 1;
-            if (!last) mbar_arrive(smem_u32(&sm.empty[at_rg.slot]));  // done with the stage
-        }
-        if (!__shfl_sync(0xffffffffu, last, kSyncLane)) return;
-        // last warp of the stage: row totals (lane = row) in a fixed order, release, rows out
-        __threadfence_block();
-        float tot = 0.f;
-        if (lane < n)
-            for (int q = 0; q < KS; ++q) tot += sp[lane * KS + q];
+    // per-stage completion: release the slot; a whole row goes out now, a slice sum to pp
+    auto finish = [&](const Ring& at_rg, int jst, int n, float part) {
         __syncwarp();
-        if (lane == kSyncLane) {
-            sm.scnt[at_rg.slot] = 0;
-            mbar_arrive(smem_u32(&sm.empty[at_rg.slot]));  // partial sums read: the slot may refill
-        }
-        if (phase == kGU) {
-            // rows come in (gate, up) pairs, lane 2j holding gate j and lane 2j + 1 up j:
-            // the FFN hidden value silu(gate) * up is formed here, once, for the D phase
-            const float up = __shfl_down_sync(0xffffffffu, tot, 1);
-            if (lane < n && (lane & 1) == 0)
-                row_out(P, sm, phase, (r0 + lane) >> 1, tot / (1.0f + expf(-tot)) * up, sc, own0);
-        } else if (lane < n) {
-            row_out(P, sm, phase, r0 + lane, tot, sc, own0);
+        if (lane == kSyncLane) mbar_arrive(smem_u32(&sm.empty[at_rg.slot]));  // done with the stage
+        if (lane == 0 && row < n) {
+            if (KS == 1) row_out(P, sm, phase, g.row0 + jst * g.R + row, part, sc, own0);
+            else pp[(jst * g.R + row) * KS + ks] = part;
         }
     };
 
@@ -683,10 +768,26 @@ __device__ __forceinline__ void run_gemv_t(const Params& P, const Smem& sm_ref, 
             if (lane == 0 && row < na) row_out(P, sm, phase, (ra0 >> 1) + row, pa / (1.0f + expf(-pa)) * pb, sc, own0);
             continue;
         }
-        finish(ra, ra0, na, pa);
-        if (two) finish(rb, rb0, nb, pb);
+        finish(ra, ja, na, pa);
+        if (two) finish(rb, jb, nb, pb);
     }
     if (threadIdx.x == 0) tr.mark(5);  // this warp's stages done
+    if (KS > 1) {
+        consumer_sync();
+        const int nrows = g.row1 - g.row0;
+        for (int i = threadIdx.x; i < nrows; i += kConsumerThreads) {
+            float tot = 0.f;
+            for (int q = 0; q < KS; ++q) tot += pp[i * KS + q];
+            if (phase != kGU) {
+                row_out(P, sm, phase, g.row0 + i, tot, sc, own0);
+            } else if ((i & 1) == 0) {
+                // interleaved (gate, up) rows: the FFN hidden value silu(gate) * up
+                float up = 0.f;
+                for (int q = 0; q < KS; ++q) up += pp[(i + 1) * KS + q];
+                row_out(P, sm, phase, (g.row0 + i) >> 1, tot / (1.0f + expf(-tot)) * up, sc, own0);
+            }
+        }
+    }
     rg_ref = rg;
     ok_ref = ok;
     // LM head: fold the lanes' running argmax into lane 0's (lowest index on ties)
@@ -769,19 +870,40 @@ __device__ __forceinline__ void run_attention(const Params& P, const Smem& sm_re
     // cache, rounded to bf16, and keeps a copy for its own pass below. Every load of this
     // prologue is issued before any store (one L2 round trip): at most 2 q pairs per thread
     // (r * HD / 2 <= 512), and one K and one V pair for threads below HD / 2.
-    const float* raw = reinterpret_cast<const float*>(P.arena + P.lay.qkv);
-    const float* qg = raw + (size_t)at.g * r * HD;
+    // The projections are tagged words written by the QKV phase (tag one below this phase's).
+    const unsigned long long* raw = reinterpret_cast<const unsigned long long*>(P.arena + P.lay.qkv);
+    const uint32_t qkv_tag = sc.tag - 1u;
+    const unsigned long long* qg = raw + (size_t)at.g * r * HD;
     const bool has_current = at.b > sc.p;
     const bool kv_lane = has_current && tid < HD / 2;
     float2 qv[2], kv2, vv2;
+    {
+        ulonglong2 wq[2], wk, wv;
+        const unsigned long long* pq[2];
+        const unsigned long long* pk = raw + dm.qd + (size_t)at.g * HD + 2 * tid;
+        const unsigned long long* pv = pk + dm.kvd;
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
-        const int t = tid + u * kConsumerThreads;
-        if (t < r * HD / 2) qv[u] = __ldcg(reinterpret_cast<const float2*>(qg + (t / (HD / 2)) * HD + 2 * (t % (HD / 2))));
-    }
-    if (kv_lane) {
-        kv2 = __ldcg(reinterpret_cast<const float2*>(raw + dm.qd + (size_t)at.g * HD + 2 * tid));
-        vv2 = __ldcg(reinterpret_cast<const float2*>(raw + dm.qd + dm.kvd + (size_t)at.g * HD + 2 * tid));
+        for (int u = 0; u < 2; ++u) {
+            const int t = tid + u * kConsumerThreads;
+            pq[u] = qg + (t / (HD / 2)) * HD + 2 * (t % (HD / 2));
+            if (t < r * HD / 2) wq[u] = ld_tagged2(pq[u]);
+        }
+        if (kv_lane) {
+            wk = ld_tagged2(pk);
+            wv = ld_tagged2(pv);
+        }
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            if (tid + u * kConsumerThreads < r * HD / 2) {
+                if (!get_pair(pq[u], qkv_tag, wq[u], P, ctl, 3)) ok = false;
+                qv[u] = make_float2(tagged_value(wq[u].x), tagged_value(wq[u].y));
+            }
+        }
+        if (kv_lane) {
+            if (!get_pair(pk, qkv_tag, wk, P, ctl, 4) || !get_pair(pv, qkv_tag, wv, P, ctl, 4)) ok = false;
+            kv2 = make_float2(tagged_value(wk.x), tagged_value(wk.y));
+            vv2 = make_float2(tagged_value(wv.x), tagged_value(wv.y));
+        }
     }
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
@@ -1001,7 +1123,8 @@ __device__ __forceinline__ void run_attention(const Params& P, const Smem& sm_re
         // batches of kCombineBatch, all loads of a batch in flight together, folding each
         // batch in with the usual max-rescaled sum (pieces in ascending order).
         const float* hp = part + (size_t)at.g * A * r * rec;
-        float* og = reinterpret_cast<float*>(const_cast<uint8_t*>(P.arena) + P.lay.o) + (size_t)at.g * r * HD;
+        unsigned long long* og = reinterpret_cast<unsigned long long*>(const_cast<uint8_t*>(P.arena) + P.lay.o) +
+                                 (size_t)at.g * r * HD;
         const size_t stride = (size_t)r * rec;
         for (int idx = tid; idx < r * HD; idx += kConsumerThreads) {
             const int h = idx / HD, dd = idx % HD;
@@ -1032,7 +1155,7 @@ __device__ __forceinline__ void run_attention(const Params& P, const Smem& sm_re
                     M = Mb;
                 }
             }
-            __stcg(og + (size_t)h * HD + dd, o / L);
+            st_tagged(og + (size_t)h * HD + dd, o / L, sc.tag);
         }
         if (tid == 0) tr.mark(7);
     }
@@ -1205,10 +1328,9 @@ struct Producer {
         uint32_t b1, b2;
         int kv_last;
         cur.stage(P, s1, b1, s2, b2, kv_last);
-        if (kv_last >= P.pos0) {  // written earlier in this launch: wait for the barrier after
-            // the attention phase (which appends the row) of the step that wrote it
-            const long long need = barriers_before_step(P, kv_last - P.pos0) + 5ll * cur.l + 2;
-            if (!wait_epochs(need)) return false;
+        if (kv_last >= P.pos0) {  // written earlier in this launch: wait for the grid barrier
+            // that ends the step that appended it (the attention phase writes the row)
+            if (!wait_epochs((long long)(kv_last - P.pos0) + 1)) return false;
         }
         if (!wait_landed()) return false;
         if (!wait_empty()) return false;
@@ -1315,7 +1437,7 @@ __global__ void __launch_bounds__(kThreads, 1) monokernel(const __grid_constant_
 
     // ---------------- consumers
     int32_t* tokens_in = reinterpret_cast<int32_t*>(const_cast<uint8_t*>(P.arena) + P.lay.tokens_in);
-    float* xg = reinterpret_cast<float*>(const_cast<uint8_t*>(P.arena) + P.lay.x);
+    const unsigned long long* tagged = reinterpret_cast<const unsigned long long*>(P.arena);
     const __nv_bfloat16* embed = reinterpret_cast<const __nv_bfloat16*>(P.arena + P.lay.embed);
     long long epoch = 0;
     Ring rg;
@@ -1360,31 +1482,35 @@ __global__ void __launch_bounds__(kThreads, 1) monokernel(const __grid_constant_
             break;
         }
         const __nv_bfloat16* erow = embed + (size_t)tok * dm.d;
-        for (int i = own0 + tid; i < own1; i += kConsumerThreads) {
-            const float v = __bfloat162float(erow[i]);
-            sm.xown[i - own0] = v;  // the residual rows this CTA updates in O and D
-            __stcg(xg + i, v);
-        }
+        for (int i = own0 + tid; i < own1; i += kConsumerThreads)
+            sm.xown[i - own0] = __bfloat162float(erow[i]);  // the residual rows this CTA updates in O and D
 
         // The step's phases in order: per layer QKV, ATT, O, GU, D, then the LM head if this
         // step's logits are needed. One loop with one call site per phase kind keeps the
-        // (fully inlined) kernel's code and register allocation to one copy of each.
+        // (fully inlined) kernel's code and register allocation to one copy of each. Every
+        // phase's input is the previous phase's tagged output (the first QKV reads the
+        // embedding row), so phases follow each other without grid barriers; one barrier
+        // ends the step (the argmax and the KV rows appended this step are then complete).
         const int nphase = 5 * dm.L + (step_has_head(P, t) ? 1 : 0);
         for (int q = 0; q < nphase; ++q) {
             const int l = q / 5 < dm.L ? q / 5 : 0;
             const int ph = q / 5 < dm.L ? q % 5 : kLM;
             sc.l = l;
+            sc.tag = phase_tag(P, t, q);
+            const uint32_t tag_in = sc.tag - 1u;  // the previous phase's
             const uint8_t* lb = P.arena + P.lay.layer0 + (size_t)l * P.lay.layer_stride;
             // this phase's input vector -> xs
             if (ph == kO) {
-                load_vector(sm, reinterpret_cast<const float*>(P.arena + P.lay.o), dm.qd);
+                load_vector(sm, tagged + P.lay.o / 8, tag_in, dm.qd, P, ctl, ok);
             } else if (ph == kD) {
-                load_vector(sm, reinterpret_cast<const float*>(P.arena + P.lay.gu), dm.F);
+                load_vector(sm, tagged + P.lay.gu / 8, tag_in, dm.F, P, ctl, ok);
             } else if (ph != kATT) {
                 const __nv_bfloat16* gain = reinterpret_cast<const __nv_bfloat16*>(
                     ph == kQKV ? lb + P.lay.l_attn_norm : ph == kGU ? lb + P.lay.l_ffn_norm : P.arena + P.lay.final_norm);
                 const bool from_embed = ph == kQKV && l == 0;
-                load_rmsnorm(sm, from_embed ? nullptr : xg, from_embed ? erow : nullptr, gain, dm.d, dm.eps);
+                const unsigned long long* xin = tagged + P.lay.x / 8 + (ph == kGU ? 0 : dm.d);  // O's or D's output
+                load_rmsnorm(sm, from_embed ? nullptr : xin, tag_in, from_embed ? erow : nullptr, gain, dm.d, dm.eps, P,
+                             ctl, ok);
             }
             if (tid == 0) tr.mark(1);
             if (ph == kATT) {
@@ -1401,7 +1527,11 @@ __global__ void __launch_bounds__(kThreads, 1) monokernel(const __grid_constant_
                     atomicMax(ctl + kCtlArgmax + 16 * (t % 3), b);
                 }
             }
-            if (!(ok = grid_sync(sm, epoch, base, P, ctl, ok, tr))) break;
+            if (q + 1 < nphase) {
+                if (!(ok = phase_end(ok, tr))) break;
+            } else {
+                if (!(ok = grid_sync(sm, epoch, base, P, ctl, ok, tr))) break;
+            }
         }
     }
     if (ok && blockIdx.x == 0 && tid == 0) {

@@ -47,7 +47,10 @@ struct Layout {
     size_t l_attn_norm, l_ffn_norm, l_wqkv, l_wo, l_wgu, l_wd;  // within a layer block
     size_t rope;                                                  // [S][hd/2] float2 (cos, sin)
     size_t kcache, vcache;                                        // [L][Hkv][S][hd] bf16
-    size_t x, qkv, o, gu, part;                                   // fp32 scratch
+    // Activations exchanged between CTAs, each element a 64-bit word (fp32 value in the low
+    // half, the producing phase's tag in the high half): x [2][d] (outputs of O and of D),
+    // qkv [qkv_rows], o [qd], gu [F] (the FFN hidden vector). Attention partials are fp32.
+    size_t x, qkv, o, gu, part;
     size_t ctl, tokens_in, tokens_out;
     size_t weights_end, kv_bytes, total;
 };
@@ -63,6 +66,15 @@ inline int rows_per_stage(int K, bool paired) {
     while (p2 * 2 <= r) p2 *= 2;
     (void)paired;
     return p2;
+}
+
+// Phases one launch runs: per step 5 per layer (QKV, ATT, O, GU, D), plus the LM head at
+// the steps that pick a token (or at every step when logits are dumped). Tags of
+// successive launches follow each other, so a buffer element never carries a stale tag
+// that a reader of a later launch expects.
+inline long long launch_phases(const Dims& dm, int steps, int n_pending, bool dump) {
+    const long long heads = dump ? steps : (steps - (n_pending - 1) > 0 ? steps - (n_pending - 1) : 0);
+    return (long long)steps * 5 * dm.L + heads;
 }
 
 struct Params {
@@ -89,6 +101,7 @@ struct Params {
     long long timeout_ns;
     int prefetch;  // stages the producer pulls into L2 ahead of the shared-memory ring
     int inflight;  // at most this many issued stages not yet landed (bounds memory queueing)
+    uint32_t tag0;  // phase i of this launch tags its outputs tag0 + 1 + i (see kd_kernel.cu)
     // optional trace: CTAs with blockIdx.x % trace_every == 0 record per-phase timestamps
     unsigned long long* trace;
     int trace_every, trace_rows;  // rows per traced CTA (4 words each)

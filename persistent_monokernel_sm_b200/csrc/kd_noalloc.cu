@@ -70,8 +70,8 @@ extern "C" int kd_decode_noalloc(kd_ctx* ctx, const int32_t* d_tokens, int32_t n
         off = up256(off + bytes);
         return at;
     };
-    const size_t o_x = take((size_t)dm.d * 4), o_q = take((size_t)dm.qkv_rows * 4), o_o = take((size_t)dm.qd * 4);
-    const size_t o_hdn = take((size_t)dm.F * 4);
+    const size_t o_x = take((size_t)2 * dm.d * 8), o_q = take((size_t)dm.qkv_rows * 8), o_o = take((size_t)dm.qd * 8);
+    const size_t o_hdn = take((size_t)dm.F * 8);
     const size_t o_part = take((size_t)v.nb * dm.r * (dm.hd + 2) * 4);
     const size_t o_ctl = take((size_t)kCtlWords * 8);
     const size_t o_tok = take((size_t)n_tokens * 4);
@@ -92,9 +92,11 @@ extern "C" int kd_decode_noalloc(kd_ctx* ctx, const int32_t* d_tokens, int32_t n
         return kd_internal_fail(ctx, KD_ECUDA, cudaGetErrorString(e));
     uint8_t* s = static_cast<uint8_t*>(base);
 
-    // Control words must start at zero (the array keeps the previous call's contents);
-    // the pending tokens are copied in. Neither allocates.
+    // Control words and the tagged activation words must start at zero (the array keeps the
+    // previous call's contents, possibly another handle's, so tags restart at 1 each call);
+    // the pending tokens are copied in. None of this allocates.
     if ((e = cudaMemsetAsync(s + o_ctl, 0, (size_t)kCtlWords * 8, (cudaStream_t)v.stream)) != cudaSuccess ||
+        (e = cudaMemsetAsync(s + o_x, 0, o_part - o_x, (cudaStream_t)v.stream)) != cudaSuccess ||
         (e = cudaMemcpyAsync(s + o_tok, d_tokens, (size_t)n_tokens * 4, cudaMemcpyDeviceToDevice, (cudaStream_t)v.stream)) !=
             cudaSuccess)
         return kd_internal_fail(ctx, KD_ECUDA, cudaGetErrorString(e));
@@ -130,6 +132,7 @@ extern "C" int kd_decode_noalloc(kd_ctx* ctx, const int32_t* d_tokens, int32_t n
     p.timeout_ns = v.timeout_ns;
     p.prefetch = v.prefetch;
     p.inflight = v.inflight;
+    p.tag0 = 0;
     int err = 0;
     launch_decode(p, v.stream, v.smem, &err);
     if (err != 0) return kd_internal_fail(ctx, KD_ECUDA, cudaGetErrorString((cudaError_t)err));
