@@ -210,9 +210,11 @@ class Decoder:
         self.pending = 0
 
     def close(self):
-        if getattr(self, "h", None):
-            kd_destroy(self.h)
+        h = getattr(self, "h", None)
+        if h:
             self.h = None
+            if kd_destroy is not None:  # None while the interpreter is shutting down
+                kd_destroy(h)
 
     __del__ = close
 

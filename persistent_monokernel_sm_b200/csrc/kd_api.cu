@@ -151,21 +151,11 @@ __global__ void repack_qkv(uint8_t* dst_layer0, size_t layer_stride, size_t off,
     for (int i = threadIdx.x; i < dm.d / 8; i += blockDim.x) d[i] = s[i];
 }
 
-// blk == 1: dst rows (2i, 2i + 1) = (gate row i, up row i). blk > 1: blocks of 2 * blk rows,
-// the gate rows of units [b * blk, (b + 1) * blk) followed by their up rows (the kernel then
-// reads a unit's gate and up rows in two consecutive stages, in the same warp).
+// dst rows (2i, 2i + 1) = (gate row i, up row i)
 __global__ void repack_gu(uint8_t* dst_layer0, size_t layer_stride, size_t off, const uint16_t* wg,
-                          const uint16_t* wu, Dims dm, int blk) {
+                          const uint16_t* wu, Dims dm) {
     const int r = blockIdx.x, l = blockIdx.y;
-    int unit, up;
-    if (blk == 1) {
-        unit = r >> 1, up = r & 1;
-    } else {
-        const int b = r / (2 * blk), w = r % (2 * blk);
-        up = w >= blk;
-        unit = b * blk + (up ? w - blk : w);
-    }
-    const uint16_t* src = (up ? wu : wg) + ((size_t)l * dm.F + unit) * dm.d;
+    const uint16_t* src = ((r & 1) ? wu : wg) + ((size_t)l * dm.F + (r >> 1)) * dm.d;
     const uint4* s = reinterpret_cast<const uint4*>(src);
     uint4* d = reinterpret_cast<uint4*>(dst_layer0 + (size_t)l * layer_stride + off + (size_t)r * dm.d * 2);
     for (int i = threadIdx.x; i < dm.d / 8; i += blockDim.x) d[i] = s[i];
@@ -257,18 +247,18 @@ int kd_create(const kd_config* cfg, void* d_arena, size_t arena_bytes, void* str
         int xs = d.d;
         if (d.qd > xs) xs = d.qd;
         if (d.F > xs) xs = d.F;
-        const int merge = kConsumerWarps * d.r * (d.hd + 2);
+        const int merge = (kConsumerWarps + 1) * d.r * (d.hd + 2);  // warps' records + the current position's
         if (merge > xs) xs = merge;
-        // GEMV phases whose rows are split over several warps keep [row][slice] sums in xs
+        // every GEMV phase keeps its [row][slice] sums in xs until the phase ends
         {
             const int K[5] = {d.d, d.qd, d.d, d.F, d.d};
             const long long units[5] = {d.qkv_rows / 2, d.d, d.F, d.d, d.V};
             const int rpu[5] = {2, 1, 2, 1, 1};
             for (int i = 0; i < 5; ++i) {
                 const int R = rows_per_stage(K[i], false);
-                if (R >= kGroupWarps) continue;
+                const int slices = R >= 2 ? 16 / R : 8;
                 const long long rows = (units[i] + c->nb - 1) / c->nb * rpu[i];
-                if (rows * (kGroupWarps / R) > xs) xs = (int)(rows * (kGroupWarps / R));
+                if (rows * slices > xs) xs = (int)(rows * slices);
             }
         }
         c->xs_floats = (xs + 31) & ~31;
@@ -286,7 +276,7 @@ int kd_create(const kd_config* cfg, void* d_arena, size_t arena_bytes, void* str
             p.ns = c->ns;
             c->smem = monokernel_smem_bytes(p);
             int per_sm = 0;
-            int e = monokernel_occupancy(d.hd, d.r, c->smem, &per_sm);
+            int e = monokernel_occupancy(d, c->smem, &per_sm);
             if (e != 0) rc = fail(c, KD_ECUDA, "occupancy query failed: %s", cudaGetErrorString((cudaError_t)e));
             else if (per_sm < 1)
                 rc = fail(c, KD_ECOOP, "monokernel cannot be resident (smem %d bytes)", c->smem);
@@ -332,9 +322,8 @@ int kd_load_weights(kd_ctx* c, const kd_weights* w) {
     repack_qkv<<<dim3(d.qkv_rows, d.L), 128, 0, s>>>(l0, y.layer_stride, y.l_wqkv, (const uint16_t*)w->wq,
                                                       (const uint16_t*)w->wk, (const uint16_t*)w->wv, d);
     KD_CUDA(c, cudaGetLastError());
-    const int gu_rows = rows_per_stage(d.d, true);
     repack_gu<<<dim3(2 * d.F, d.L), 128, 0, s>>>(l0, y.layer_stride, y.l_wgu, (const uint16_t*)w->wg,
-                                                  (const uint16_t*)w->wu, d, gu_rows == kGroupWarps ? gu_rows : 1);
+                                                  (const uint16_t*)w->wu, d);
     KD_CUDA(c, cudaGetLastError());
     c->launches += 2;
     // RoPE table: (cos, sin) of position p times frequency theta^(-2i/hd), formed in double

@@ -183,6 +183,13 @@ struct Gemv {
     int nst;              // stages
 };
 
+// log2 of the slices per row of a GEMV stage with R rows: 16 / R for R >= 2, 8 for R == 1
+// (R is a power of two <= 8; see run_gemv_t).
+__device__ __forceinline__ int gemv_log_slices(int R) {
+    const int lr = __ffs(R) - 1;
+    return R >= 2 ? 4 - lr : 3;
+}
+
 // This CTA's rows of every GEMV phase, [phase][row0, row1, stages], and the residual rows
 // it owns: computed once per launch into shared memory (the 64-bit divisions that split the
 // rows over the grid would otherwise be paid by every warp at every phase).
@@ -194,11 +201,7 @@ __device__ void cta_geometry(const Params& P, int c, int* geom) {
         switch (phase) {
             case kQKV: units = dm.qkv_rows / 2; rpu = 2; R = P.rows_qkv; break;
             case kO: units = dm.d; R = P.rows_o; break;
-            case kGU:  // blocks of R gate rows then R up rows when a warp owns a row, else pairs
-                R = P.rows_gu;
-                if (R == kGroupWarps) units = dm.F / R, rpu = 2 * R;
-                else units = dm.F, rpu = 2;
-                break;
+            case kGU: units = dm.F; rpu = 2; R = P.rows_gu; break;  // (gate, up) row pairs
             case kD: units = dm.d; R = P.rows_d; break;
             case kLM: units = dm.V; R = P.rows_lm; break;
             default: break;
@@ -237,6 +240,7 @@ struct Attn {
     int nst;       // ring stages of the piece
 };
 
+constexpr int kLastPieceRelief = 64;
 __device__ __forceinline__ Attn attn_geom(const Params& P, int p, int c) {
     Attn at;
     const int A = P.attn_pieces;
@@ -248,9 +252,19 @@ __device__ __forceinline__ Attn attn_geom(const Params& P, int p, int c) {
     }
     at.g = c / A;
     at.piece = c % A;
+    // The last piece also appends the current position, folds it in and usually combines the
+    // head's pieces, so it takes kLastPieceRelief fewer cached positions than an even share;
+    // the other pieces split the rest evenly.
     const long long T = (long long)p + 1;
-    at.a = (int)(T * at.piece / A);
-    at.b = (int)(T * (at.piece + 1) / A);
+    long long last = T / A - kLastPieceRelief;
+    if (last < 1 || A == 1) last = A == 1 ? T : 1;
+    if (at.piece == A - 1) {
+        at.a = (int)(T - last);
+        at.b = (int)T;
+    } else {
+        at.a = (int)((T - last) * at.piece / (A - 1));
+        at.b = (int)((T - last) * (at.piece + 1) / (A - 1));
+    }
     at.tma_end = at.b < p ? at.b : p;
     if (at.tma_end < at.a) at.tma_end = at.a;
     at.nst = (at.tma_end - at.a + P.pos_per_stage - 1) / P.pos_per_stage;
@@ -630,22 +644,20 @@ __device__ __forceinline__ void row_out(const Params& P, const Smem& sm, int pha
     }
 }
 
-// One GEMV phase. Consumer groups take the stages of their ring slots (slot mod kGroups).
-// Within a group the R (<= 8) rows of a stage are split over its 8 warps as R rows x 8/R
-// slices of the reduction dimension; a warp keeps its slice of the activation vector in
-// registers for the whole phase, so a stage costs it one 16-byte shared-memory load and 8
-// FMAs per chunk. When a warp owns a whole row (R = 8) it finishes the row itself; when rows
-// are split, the warps' partial sums meet in shared memory and the last warp of the stage
-// adds them in a fixed order. Either way the per-row epilogue (row_out) is a store or two.
-// A wait that gives up marks `ok` false and the warp skips the work of the remaining
-// stages, but it still reaches every named barrier; the next grid barrier then reports
-// the failure to the whole CTA at once.
-//
-// NCL > 0: every warp's slice is exactly NCL chunks per lane, so the chunk loop has no
-// per-lane bounds test and its shared-memory addresses are one base plus constants (this
-// is the case for every shape whose reduction length is a multiple of 256 x slices). NCL = 0
-// is the general case (any multiple of 64), with a per-chunk test.
-template <int NCL>
+// One GEMV phase. A stage holds R rows (R a power of two <= 8); each row is cut into KS
+// slices of the reduction dimension and the 8 warps share the R * KS (row, slice) units:
+//   R >= 2: KS = 16 / R, 16 units, warp w takes units w and w + 8 -- the same slice of two
+//           rows R / 2 apart, so one activation slice in registers serves both;
+//   R == 1: KS = 8, warp w takes slice w of the one row.
+// The slice is at most 1024 elements when R >= 2 (4 chunks of 8 per lane), which keeps the
+// kernel's register demand low enough to avoid spilling. A warp's slice sums go to xs (free
+// once every warp holds its activation slice) as [local row][slice]; after the last stage
+// the rows are summed in slice order and put out (row_out), the gate/up rows in pairs.
+// NCL > 0: every slice is exactly NCL chunks per lane, so the chunk loop has no bounds test.
+// A wait that gives up marks `ok` false and the warp skips the work of the remaining stages,
+// but it still reaches every named barrier; the phase end then reports the failure to the
+// whole CTA at once.
+template <int NCL, int MAXCH>
 __device__ __forceinline__ void run_gemv_t(const Params& P, const Smem& sm_ref, unsigned long long* ctl, int phase, int l,
                                         Ring& rg_ref, StepCtx& sc_ref, bool& ok_ref, Tracer& tr) {
     const Smem sm = sm_ref;
@@ -656,18 +668,18 @@ __device__ __forceinline__ void run_gemv_t(const Params& P, const Smem& sm_ref, 
     const int nst = g.nst;
     const int ns = P.ns;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int group = warp / kGroupWarps, gw = warp % kGroupWarps;
-    // slices per row: rows_per_stage gives R in {1, 2, 4, 8}, so KS is a power of two too
-    const int lks = 3 - (__ffs(g.R) - 1), KS = 1 << lks;
-    const int row = gw >> lks, ks = gw & (KS - 1);
+    const bool dual = g.R >= 2;
+    const int lks = gemv_log_slices(g.R), KS = 1 << lks;  // slices per row
+    const int ks = warp & (KS - 1);                        // this warp's slice
+    const int rowa = warp >> lks, rowb = (warp + 8) >> lks;  // its rows within a stage
     const int nch = g.K >> 3;
     const int c0 = (nch * ks) >> lks, c1 = (nch * (ks + 1)) >> lks;  // at most 32 * kMaxChunks chunks
-    const size_t rowb = (size_t)g.K * 2;
+    const size_t rowbytes = (size_t)g.K * 2;
     const int own0 = sm.geom[kGeomOwn];
     unsigned long long& waited = tr.waited;
 
     // this lane's activation chunks: c = c0 + lane + 32 i
-    constexpr int NX = NCL > 0 ? NCL : kMaxChunks;
+    constexpr int NX = NCL > 0 ? NCL : MAXCH;
     float xr[NX][8];
     const float4* xlo = reinterpret_cast<const float4*>(sm.xs);
     const float4* xhi = reinterpret_cast<const float4*>(sm.xs + (g.K >> 1));
@@ -681,15 +693,10 @@ __device__ __forceinline__ void run_gemv_t(const Params& P, const Smem& sm_ref, 
         xr[i][4] = b.x, xr[i][5] = b.y, xr[i][6] = b.z, xr[i][7] = b.w;
     }
     if (threadIdx.x == 0) tr.mark(7);  // activation slice in registers
-    // When rows are split over KS > 1 warps, each warp's slice sums go to xs (free once every
-    // warp holds its activation slice) as [local row][slice] and are added up, in slice order,
-    // when the phase's stages are done: no per-stage cross-warp handshake.
     float* pp = sm.xs;
-    if (KS > 1) consumer_sync();
+    consumer_sync();  // every warp has its slice: xs now takes the slice sums
 
-    // Stages are taken two at a time (this group's next two): their 16 chunk loads and the
-    // two cross-lane reductions interleave, and the per-stage bookkeeping is paid once per pair.
-    auto dot_row = [&](const uint8_t* wrow, float& s) {
+    auto dot_row = [&](const uint8_t* wrow) {
         float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
         const uint8_t* wl = wrow + (c0 + lane) * 16;  // this lane's first chunk; then +512 B each
 #pragma unroll
@@ -706,86 +713,65 @@ __device__ __forceinline__ void run_gemv_t(const Params& P, const Smem& sm_ref, 
                 a3 = fmaf(bf_hi(w.w), xr[i][7], a3);
             }
         }
-        s = (a0 + a1) + (a2 + a3);
-    };
-    // per-stage completion: release the slot; a whole row goes out now, a slice sum to pp
-    auto finish = [&](const Ring& at_rg, int jst, int n, float part) {
-        __syncwarp();
-        if (lane == kSyncLane) mbar_arrive(smem_u32(&sm.empty[at_rg.slot]));  // done with the stage
-        if (lane == 0 && row < n) {
-            if (KS == 1) row_out(P, sm, phase, g.row0 + jst * g.R + row, part, sc, own0);
-            else pp[(jst * g.R + row) * KS + ks] = part;
-        }
+        return (a0 + a1) + (a2 + a3);
     };
 
-    int j = 0;
-    while (j < nst) {
-        // this group's next stage, and the one after it
-        while (j < nst && rg.slot % kGroups != group) {
-            ++j;
-            rg.advance(ns);
-        }
-        if (j >= nst) break;
-        const int ja = j;
+    // Stages are taken two at a time: the four dot products (two rows of each stage) and their
+    // reductions interleave, and the per-stage bookkeeping is paid once per pair.
+    auto put = [&](int j, int n, float pa, float pb) {
+        if (rowa < n) pp[(j * g.R + rowa) * KS + ks] = pa;
+        if (dual && rowb < n) pp[(j * g.R + rowb) * KS + ks] = pb;
+    };
+    for (int j = 0; j < nst; j += 2) {
         const Ring ra = rg;
-        ++j;
         rg.advance(ns);
-        while (j < nst && rg.slot % kGroups != group) {
-            ++j;
-            rg.advance(ns);
-        }
-        const bool two = j < nst;
-        const int jb = j;
+        const bool two = j + 1 < nst;
         const Ring rb = rg;
-        if (two) {
-            ++j;
-            rg.advance(ns);
-        }
+        if (two) rg.advance(ns);
         if (!ok) continue;
         if (!wait_full(sm, ra, P, ctl, waited) || (two && !wait_full(sm, rb, P, ctl, waited))) {
             ok = false;
             continue;
         }
-        if (threadIdx.x == 0 && ja == 0) tr.mark(4);  // first stage of the phase ready
-        const int ra0 = g.row0 + ja * g.R, na = min(g.R, g.row1 - ra0);
-        const int rb0 = g.row0 + jb * g.R, nb = two ? min(g.R, g.row1 - rb0) : 0;
-        float pa = 0.f, pb = 0.f;
-        if (row < na) dot_row(sm.ring + (size_t)ra.slot * kStageBytes + row * rowb, pa);
-        if (row < nb) dot_row(sm.ring + (size_t)rb.slot * kStageBytes + row * rowb, pb);
+        if (threadIdx.x == 0 && j == 0) tr.mark(4);  // first stage of the phase ready
+        const int na = min(g.R, g.row1 - (g.row0 + j * g.R));            // rows in stage j
+        const int nb = two ? min(g.R, g.row1 - (g.row0 + (j + 1) * g.R)) : 0;  // rows in stage j + 1
+        const uint8_t* sa = sm.ring + (size_t)ra.slot * kStageBytes;
+        const uint8_t* sb = sm.ring + (size_t)rb.slot * kStageBytes;
+        float p0 = rowa < na ? dot_row(sa + rowa * rowbytes) : 0.f;
+        float p1 = dual && rowb < na ? dot_row(sa + rowb * rowbytes) : 0.f;
+        float p2 = rowa < nb ? dot_row(sb + rowa * rowbytes) : 0.f;
+        float p3 = dual && rowb < nb ? dot_row(sb + rowb * rowbytes) : 0.f;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
-            pa += __shfl_xor_sync(0xffffffffu, pa, o);
-            pb += __shfl_xor_sync(0xffffffffu, pb, o);
+            p0 += __shfl_xor_sync(0xffffffffu, p0, o);
+            p1 += __shfl_xor_sync(0xffffffffu, p1, o);
+            p2 += __shfl_xor_sync(0xffffffffu, p2, o);
+            p3 += __shfl_xor_sync(0xffffffffu, p3, o);
         }
-        if (phase == kGU && KS == 1) {
-            // block layout: stage a holds R gate rows, stage b the R up rows of the same units,
-            // so this warp has both halves of its unit and forms silu(gate) * up itself
-            __syncwarp();
-            if (lane == kSyncLane) {
-                mbar_arrive(smem_u32(&sm.empty[ra.slot]));
-                mbar_arrive(smem_u32(&sm.empty[rb.slot]));
-            }
-            if (lane == 0 && row < na) row_out(P, sm, phase, (ra0 >> 1) + row, pa / (1.0f + expf(-pa)) * pb, sc, own0);
-            continue;
+        __syncwarp();
+        if (lane == kSyncLane) {  // done with the stages
+            mbar_arrive(smem_u32(&sm.empty[ra.slot]));
+            if (two) mbar_arrive(smem_u32(&sm.empty[rb.slot]));
         }
-        finish(ra, ja, na, pa);
-        if (two) finish(rb, jb, nb, pb);
+        if (lane == 0) {
+            put(j, na, p0, p1);
+            if (two) put(j + 1, nb, p2, p3);
+        }
     }
     if (threadIdx.x == 0) tr.mark(5);  // this warp's stages done
-    if (KS > 1) {
-        consumer_sync();
-        const int nrows = g.row1 - g.row0;
-        for (int i = threadIdx.x; i < nrows; i += kConsumerThreads) {
-            float tot = 0.f;
-            for (int q = 0; q < KS; ++q) tot += pp[i * KS + q];
-            if (phase != kGU) {
-                row_out(P, sm, phase, g.row0 + i, tot, sc, own0);
-            } else if ((i & 1) == 0) {
-                // interleaved (gate, up) rows: the FFN hidden value silu(gate) * up
-                float up = 0.f;
-                for (int q = 0; q < KS; ++q) up += pp[(i + 1) * KS + q];
-                row_out(P, sm, phase, (g.row0 + i) >> 1, tot / (1.0f + expf(-tot)) * up, sc, own0);
-            }
+    consumer_sync();
+    const int nrows = g.row1 - g.row0;
+    for (int i = threadIdx.x; i < nrows; i += kConsumerThreads) {
+        float tot = 0.f;
+        for (int q = 0; q < KS; ++q) tot += pp[i * KS + q];
+        if (phase != kGU) {
+            row_out(P, sm, phase, g.row0 + i, tot, sc, own0);
+        } else if ((i & 1) == 0) {
+            // interleaved (gate, up) rows: the FFN hidden value silu(gate) * up
+            float up = 0.f;
+            for (int q = 0; q < KS; ++q) up += pp[(i + 1) * KS + q];
+            row_out(P, sm, phase, (g.row0 + i) >> 1, tot / (1.0f + expf(-tot)) * up, sc, own0);
         }
     }
     rg_ref = rg;
@@ -804,24 +790,28 @@ __device__ __forceinline__ void run_gemv_t(const Params& P, const Smem& sm_ref, 
 
 // Chunks (8 elements) per lane of every warp's slice when that count is exact, else 0.
 __device__ __forceinline__ int gemv_exact_chunks(int K, int R) {
-    const int lks = 3 - (__ffs(R) - 1);  // log2(kGroupWarps / R)
+    const int lks = gemv_log_slices(R);
     const int nch = K >> 3, per = nch >> (5 + lks);
     return (per << (5 + lks)) == nch && per <= kMaxChunks ? per : 0;
 }
 
+// MAXCH (4 or 8): the most chunks per lane any phase of this model needs; the kernel is
+// instantiated per MAXCH so that a model whose slices fit in 4 chunks never carries the
+// registers of an 8-chunk loop.
+template <int MAXCH>
 __device__ __forceinline__ void run_gemv(const Params& P, const Smem& sm, unsigned long long* ctl, int phase, int l,
-                                      Ring& rg, StepCtx& sc, bool& ok, Tracer& tr) {
+                                         Ring& rg, StepCtx& sc, bool& ok, Tracer& tr) {
     const Gemv g = gemv_geom(P, sm.geom, phase, l);
     switch (gemv_exact_chunks(g.K, g.R)) {
-        case 1: run_gemv_t<1>(P, sm, ctl, phase, l, rg, sc, ok, tr); break;
-        case 2: run_gemv_t<2>(P, sm, ctl, phase, l, rg, sc, ok, tr); break;
-        case 3: run_gemv_t<3>(P, sm, ctl, phase, l, rg, sc, ok, tr); break;
-        case 4: run_gemv_t<4>(P, sm, ctl, phase, l, rg, sc, ok, tr); break;
-        case 5: run_gemv_t<5>(P, sm, ctl, phase, l, rg, sc, ok, tr); break;
-        case 6: run_gemv_t<6>(P, sm, ctl, phase, l, rg, sc, ok, tr); break;
-        case 7: run_gemv_t<7>(P, sm, ctl, phase, l, rg, sc, ok, tr); break;
-        case 8: run_gemv_t<8>(P, sm, ctl, phase, l, rg, sc, ok, tr); break;
-        default: run_gemv_t<0>(P, sm, ctl, phase, l, rg, sc, ok, tr); break;
+        case 1: run_gemv_t<1, MAXCH>(P, sm, ctl, phase, l, rg, sc, ok, tr); break;
+        case 2: run_gemv_t<2, MAXCH>(P, sm, ctl, phase, l, rg, sc, ok, tr); break;
+        case 3: run_gemv_t<3, MAXCH>(P, sm, ctl, phase, l, rg, sc, ok, tr); break;
+        case 4: run_gemv_t<4, MAXCH>(P, sm, ctl, phase, l, rg, sc, ok, tr); break;
+        case 5: if constexpr (MAXCH >= 5) run_gemv_t<5, MAXCH>(P, sm, ctl, phase, l, rg, sc, ok, tr); break;
+        case 6: if constexpr (MAXCH >= 6) run_gemv_t<6, MAXCH>(P, sm, ctl, phase, l, rg, sc, ok, tr); break;
+        case 7: if constexpr (MAXCH >= 7) run_gemv_t<7, MAXCH>(P, sm, ctl, phase, l, rg, sc, ok, tr); break;
+        case 8: if constexpr (MAXCH >= 8) run_gemv_t<8, MAXCH>(P, sm, ctl, phase, l, rg, sc, ok, tr); break;
+        default: run_gemv_t<0, MAXCH>(P, sm, ctl, phase, l, rg, sc, ok, tr); break;
     }
 }
 
@@ -847,7 +837,7 @@ __device__ __forceinline__ void ld_v(const __nv_bfloat16* p, bool global, float 
 // all lanes accumulate the 8 V rows (each lane hd/32 output dims). States of the warps are
 // merged per CTA; the last CTA of a kv head to finish combines all pieces.
 // GMAX >= the number of q heads per kv head (2, 4 or 8).
-constexpr int kCombineBatch = 12;  // pieces whose records one combining thread loads at once
+constexpr int kCombineBatch = 18;  // pieces whose records one combining thread loads at once
 template <int HD, int GMAX>
 __device__ __forceinline__ void run_attention(const Params& P, const Smem& sm_ref, unsigned long long* ctl, int l,
                                           Ring& rg_ref, StepCtx& sc_ref, bool& ok_ref, Tracer& tr) {
@@ -929,9 +919,33 @@ __device__ __forceinline__ void run_attention(const Params& P, const Smem& sm_re
         *reinterpret_cast<__nv_bfloat162*>(vc + 2 * i) = v01;
         *reinterpret_cast<__nv_bfloat162*>(&sm.kvcur[HD + 2 * i]) = v01;
     }
-    if (has_current) fence_proxy_async_global();  // later bulk copies (async proxy) read these rows
+    // (Bulk copies read these rows at later steps only, after the step's grid barrier; the
+    // producer issues the proxy fence after acquiring that barrier.)
     consumer_sync();
     if (tid == 0) tr.mark(4);
+
+    // The current position's state is one record next to the warps' (slot kConsumerWarps of
+    // the merge area): score s = q . k_cur, weight sum 1, accumulator v_cur. One warp forms it
+    // before the pass over the cache, instead of a whole extra pass at the end.
+    const int rec = HD + 2;
+    float* ws = sm.xs;  // [warp][h][rec] merge area (xs is free during attention)
+    if (has_current && warp == kConsumerWarps - 1) {
+#pragma unroll
+        for (int h = 0; h < GMAX; ++h) {
+            if (h < r) {
+                float sdot = 0.f;
+#pragma unroll
+                for (int e = 0; e < E; ++e)
+                    sdot = fmaf(sm.qs[h * HD + lane * E + e], __bfloat162float(sm.kvcur[lane * E + e]), sdot);
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) sdot += __shfl_xor_sync(0xffffffffu, sdot, o);
+                float* wr = ws + ((size_t)kConsumerWarps * r + h) * rec;
+                if (lane == 0) wr[0] = sdot, wr[1] = 1.f;
+#pragma unroll
+                for (int e = 0; e < E; ++e) wr[2 + lane * E + e] = __bfloat162float(sm.kvcur[HD + lane * E + e]);
+            }
+        }
+    }
 
     float m[GMAX], lsum[GMAX], acc[GMAX][E];
 #pragma unroll
@@ -1073,13 +1087,8 @@ __device__ __forceinline__ void run_attention(const Params& P, const Smem& sm_re
         }
         j += two ? 2 : 1;
     }
-    // the current position, appended above
-    if (has_current && warp == kConsumerWarps - 1) pass2(sm.kvcur, sm.kvcur + HD, 1, sm.kvcur, sm.kvcur + HD, 0, false);
-
-    // merge the warps' states (xs is free during attention)
+    // merge the warps' states (and the current position's record)
     if (tid == 0) tr.mark(5);
-    const int rec = HD + 2;
-    float* ws = sm.xs;  // [warp][h][rec]
 #pragma unroll
     for (int h = 0; h < GMAX; ++h) {
         if (h < r) {
@@ -1092,13 +1101,14 @@ __device__ __forceinline__ void run_attention(const Params& P, const Smem& sm_re
     consumer_sync();
     float* part = reinterpret_cast<float*>(const_cast<uint8_t*>(P.arena) + P.lay.part);
     float* mine = part + ((size_t)(at.g * A + at.piece) * r) * rec;
+    const int nrec = kConsumerWarps + (has_current ? 1 : 0);
     for (int idx = tid; idx < r * HD; idx += kConsumerThreads) {
         const int h = idx / HD, dd = idx % HD;
         float M = -INFINITY;
-        for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, ws[((size_t)w * r + h) * rec]);
+        for (int w = 0; w < nrec; ++w) M = fmaxf(M, ws[((size_t)w * r + h) * rec]);
         float L = 0.f, o = 0.f;
         if (M != -INFINITY) {
-            for (int w = 0; w < kConsumerWarps; ++w) {
+            for (int w = 0; w < nrec; ++w) {
                 const float* wr = ws + ((size_t)w * r + h) * rec;
                 if (wr[0] == -INFINITY) continue;
                 const float f = exp2f(wr[0] - M);
@@ -1399,7 +1409,7 @@ struct Producer {
 
 // One instantiation per attention shape (head dim, q heads per kv head rounded up to 2, 4
 // or 8), so the fully inlined kernel holds one attention body and its registers.
-template <int HD, int GMAX>
+template <int HD, int GMAX, int MAXCH>
 __global__ void __launch_bounds__(kThreads, 1) monokernel(const __grid_constant__ Params P) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const Smem sm = carve(P, smem_raw);
@@ -1516,7 +1526,7 @@ __global__ void __launch_bounds__(kThreads, 1) monokernel(const __grid_constant_
             if (ph == kATT) {
                 run_attention<HD, GMAX>(P, sm, ctl, l, rg, sc, ok, tr);
             } else {
-                run_gemv(P, sm, ctl, ph, l, rg, sc, ok, tr);
+                run_gemv<MAXCH>(P, sm, ctl, ph, l, rg, sc, ok, tr);
             }
             if (ph == kLM) {
                 if ((tid & 31) == 0) sm.best[tid >> 5] = sc.lm_best;
@@ -1548,19 +1558,23 @@ __global__ void __launch_bounds__(kThreads, 1) monokernel(const __grid_constant_
 
 // ------------------------------------------------------------------ host-side launch
 
-static const void* kernel_for(int hd, int r) {
+template <int MAXCH>
+static const void* kernel_for_ch(int hd, int r) {
     if (hd == 128) {
-        if (r <= 2) return (const void*)monokernel<128, 2>;
-        if (r <= 4) return (const void*)monokernel<128, 4>;
-        return (const void*)monokernel<128, 8>;
+        if (r <= 2) return (const void*)monokernel<128, 2, MAXCH>;
+        if (r <= 4) return (const void*)monokernel<128, 4, MAXCH>;
+        return (const void*)monokernel<128, 8, MAXCH>;
     }
-    if (r <= 2) return (const void*)monokernel<64, 2>;
-    if (r <= 4) return (const void*)monokernel<64, 4>;
-    return (const void*)monokernel<64, 8>;
+    if (r <= 2) return (const void*)monokernel<64, 2, MAXCH>;
+    if (r <= 4) return (const void*)monokernel<64, 4, MAXCH>;
+    return (const void*)monokernel<64, 8, MAXCH>;
+}
+static const void* kernel_for(const Dims& dm) {
+    return gemv_max_chunks(dm) <= 4 ? kernel_for_ch<4>(dm.hd, dm.r) : kernel_for_ch<8>(dm.hd, dm.r);
 }
 
-int monokernel_occupancy(int hd, int r, int smem_bytes, int* blocks_per_sm) {
-    const void* k = kernel_for(hd, r);
+int monokernel_occupancy(const Dims& dm, int smem_bytes, int* blocks_per_sm) {
+    const void* k = kernel_for(dm);
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
     if (e != cudaSuccess) return (int)e;
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, k, kThreads, smem_bytes);
@@ -1569,7 +1583,7 @@ int monokernel_occupancy(int hd, int r, int smem_bytes, int* blocks_per_sm) {
 
 void launch_decode(const Params& p, void* stream, int smem_bytes, int* err) {
     void* args[] = {const_cast<Params*>(&p)};
-    cudaError_t e = cudaLaunchCooperativeKernel(kernel_for(p.dm.hd, p.dm.r), dim3(p.nb), dim3(kThreads), args,
+    cudaError_t e = cudaLaunchCooperativeKernel(kernel_for(p.dm), dim3(p.nb), dim3(kThreads), args,
                                                 (size_t)smem_bytes, (cudaStream_t)stream);
     *err = (int)e;
 }

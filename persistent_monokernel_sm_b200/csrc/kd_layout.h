@@ -56,9 +56,8 @@ struct Layout {
 };
 
 // Rows per pipeline stage of one GEMV phase with reduction length K (bf16 elements): the
-// largest power of two <= 8 whose rows fit a stage. A group of 8 warps then splits the
-// stage exactly as R rows x 8/R slices, each slice at most 2048 elements (8 chunks per
-// lane). Paired phases (RoPE pairs, gate/up pairs) always get R >= 2 since K <= 8192.
+// largest power of two <= 8 whose rows fit a stage. The kernel cuts each row into slices
+// (16 / R of them when R >= 2, else 8) shared by the 8 consumer warps.
 inline int rows_per_stage(int K, bool paired) {
     int r = kStageBytes / (2 * K);
     if (r > kMaxRows) r = kMaxRows;
@@ -66,6 +65,20 @@ inline int rows_per_stage(int K, bool paired) {
     while (p2 * 2 <= r) p2 *= 2;
     (void)paired;
     return p2;
+}
+
+// Chunks of 8 elements per lane that a GEMV slice of reduction length K needs when a stage
+// holds R = rows_per_stage(K) rows cut into 16 / R slices (R >= 2) or 8 slices (R == 1).
+inline int gemv_slice_chunks(int K) {
+    const int R = rows_per_stage(K, false);
+    const int slices = R >= 2 ? 16 / R : 8;
+    return (K / slices + 255) / 256;
+}
+inline int gemv_max_chunks(const Dims& dm) {
+    int m = gemv_slice_chunks(dm.d);
+    if (gemv_slice_chunks(dm.qd) > m) m = gemv_slice_chunks(dm.qd);
+    if (gemv_slice_chunks(dm.F) > m) m = gemv_slice_chunks(dm.F);
+    return m;
 }
 
 // Phases one launch runs: per step 5 per layer (QKV, ATT, O, GU, D), plus the LM head at
@@ -128,6 +141,6 @@ struct kd_ctx_view {
     bool has_weights;
 };
 int monokernel_smem_bytes(const Params& p);
-int monokernel_occupancy(int hd, int r, int smem_bytes, int* blocks_per_sm);
+int monokernel_occupancy(const Dims& dm, int smem_bytes, int* blocks_per_sm);
 
 }  // namespace kd
