@@ -31,7 +31,28 @@ sys.path.insert(0, ROOT)
 
 METRIC = "batch-1 decode tokens/s on 1 B200 (2B bf16) and % of HBM-bandwidth roofline"
 SPEC_HBM_GBS = 8000.0          # B200 HBM3e specification
+# DRAM bytes per algorithmic byte of the monokernel, from one ncu capture
+# (dram__bytes_read.sum + dram__bytes_write.sum of one launch decoding 8 tokens of the 2B model
+# at a 4k context; profiles/monokernel_2b-4k_8tok_counters.md). It holds for the kernel source
+# it was taken on only: when csrc/kd_kernel.cu no longer has this SHA-256, traffic is null.
+TRAFFIC_CAPTURE = {"kernel_sha256": None, "dram_bytes": None, "algorithmic_bytes": None}
 FALLBACK_HBM_GBS = 6650.0       # earlier measurement on this machine, if no measured peaks file
+
+
+def kernel_source_sha256() -> str:
+    import hashlib
+    path = os.path.join(ROOT, "persistent_monokernel_sm_b200", "csrc", "kd_kernel.cu")
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()
+
+
+def launch_traffic(bytes_launch: float):
+    """DRAM bytes of one timed launch: the captured DRAM/algorithmic ratio times this launch's
+    algorithmic bytes, or None when the kernel changed since the capture."""
+    cap = TRAFFIC_CAPTURE
+    if not cap["kernel_sha256"] or cap["kernel_sha256"] != kernel_source_sha256():
+        return None
+    return cap["dram_bytes"] / cap["algorithmic_bytes"] * bytes_launch
 
 
 def parse():
@@ -294,6 +315,7 @@ def main():
     mean_kern_ms = statistics.mean(kern_ms)
     achieved = bytes_launch / (mean_kern_ms * 1e-3) / 1e9
     peak, peak_kind = measured_peaks()
+    traffic = launch_traffic(bytes_launch)
 
     line = None
     if rank == 0:
@@ -305,7 +327,7 @@ def main():
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "storage": "bf16 weights and KV cache",
             "data": "synthetic", "config": workload_config(w, w.n_gen),
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                         "frac": achieved / peak, "traffic": None,
+                         "frac": achieved / peak, "traffic": traffic,
                          "peak_source": "%s copy bandwidth (MEASURED_PEAKS.json hbm_gbs)" % peak_kind
                          if peak_kind == "measured" else "fallback 6.65 TB/s",
                          "frac_of_8tbs_spec": achieved / SPEC_HBM_GBS,

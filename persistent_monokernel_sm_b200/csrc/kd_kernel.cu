@@ -166,6 +166,9 @@ struct Tracer {
     }
 };
 
+// 64-bit slots of the shared-memory flag words (sm.flag, 16 ints): the barrier counter base
+// and the grid barriers done (thread 0 only); ints 0-3 are broadcast slots.
+constexpr int kFlagBase = 4, kFlagEpoch = 5;
 // Lane that performs a warp's shared-memory bookkeeping (see run_gemv).
 constexpr int kSyncLane = 31;
 static_assert(kGroupWarps == 8, "GEMV slice arithmetic assumes 8 warps per group");
@@ -466,8 +469,10 @@ __device__ __forceinline__ bool get_pair(const unsigned long long* p, uint32_t t
 // `local_ok` is false in a warp whose wait gave up; the result is the same for every
 // consumer thread of the CTA, and false in every CTA once any wait anywhere has given up
 // (the device status word is re-read after the barrier completes).
-__device__ __forceinline__ bool grid_sync(const Smem& sm, long long& epoch, uint64_t base, const Params& P,
-                          unsigned long long* ctl, bool local_ok, Tracer& tr) {
+// The counter base of this launch and the barriers done so far live in shared memory
+// (kFlagBase, kFlagEpoch): only thread 0 uses them, so no thread carries them in registers.
+__device__ __forceinline__ bool grid_sync(const Smem& sm, const Params& P, unsigned long long* ctl, bool local_ok,
+                                          Tracer& tr) {
     // every consumer warp's writes of this phase are done; did every warp succeed?
     const bool cta_ok = consumer_sync_and(local_ok);
     if (threadIdx.x == 0) tr.mark(2);
@@ -478,7 +483,10 @@ __device__ __forceinline__ bool grid_sync(const Smem& sm, long long& epoch, uint
         // writes visible to this thread, and the CTA barrier after it to the others. Loads
         // of data written during the launch bypass L1 (ld.global.cg), so no fence is needed.
         red_release_add_u64(ctl + kCtlBar, 1ull);
-        const uint64_t target = base + (uint64_t)(epoch + 1) * (uint64_t)P.nb;
+        unsigned long long* bs = reinterpret_cast<unsigned long long*>(sm.flag);
+        const long long epoch = (long long)bs[kFlagEpoch];
+        bs[kFlagEpoch] = (unsigned long long)(epoch + 1);
+        const uint64_t target = bs[kFlagBase] + (uint64_t)(epoch + 1) * (uint64_t)P.nb;
         int ok = 1;
         if (ld_acquire_u64(ctl + kCtlBar) < target) {
             const uint64_t t0 = globaltimer();
@@ -501,7 +509,6 @@ __device__ __forceinline__ bool grid_sync(const Smem& sm, long long& epoch, uint
         tr.mark(0);
     }
     consumer_sync();
-    ++epoch;
     return sm.flag[0] != 0;
 }
 
@@ -1428,12 +1435,13 @@ __global__ void __launch_bounds__(kThreads, 1) monokernel(const __grid_constant_
         // Barrier count at launch: a multiple of nb plus arrivals of CTAs that already
         // reached this launch's first barrier (which cannot complete before we arrive).
         const uint64_t raw = ld_acquire_u64(ctl + kCtlBar);
-        reinterpret_cast<unsigned long long*>(sm.flag)[1] = raw - raw % (uint64_t)P.nb;
+        reinterpret_cast<unsigned long long*>(sm.flag)[kFlagBase] = raw - raw % (uint64_t)P.nb;
+        reinterpret_cast<unsigned long long*>(sm.flag)[kFlagEpoch] = 0ull;
         sm.flag[0] = read_status(ctl);
         if (blockIdx.x == 0) ctl[kCtlArgmax] = 0ull;  // step 0's argmax slot
     }
     __syncthreads();
-    const uint64_t base = reinterpret_cast<unsigned long long*>(sm.flag)[1];
+    const uint64_t base = reinterpret_cast<unsigned long long*>(sm.flag)[kFlagBase];
     if (sm.flag[0] != 0) return;  // an earlier launch failed: refuse until reset
     __syncthreads();
 
@@ -1449,7 +1457,6 @@ __global__ void __launch_bounds__(kThreads, 1) monokernel(const __grid_constant_
     int32_t* tokens_in = reinterpret_cast<int32_t*>(const_cast<uint8_t*>(P.arena) + P.lay.tokens_in);
     const unsigned long long* tagged = reinterpret_cast<const unsigned long long*>(P.arena);
     const __nv_bfloat16* embed = reinterpret_cast<const __nv_bfloat16*>(P.arena + P.lay.embed);
-    long long epoch = 0;
     Ring rg;
     StepCtx sc;
     bool ok = true;
@@ -1459,7 +1466,6 @@ __global__ void __launch_bounds__(kThreads, 1) monokernel(const __grid_constant_
         tr.rows = P.trace_rows;
         tr.mark(0);
     }
-    const int own0 = sm.geom[kGeomOwn], own1 = sm.geom[kGeomOwn + 1];
 
     for (int t = 0; t < P.steps && ok; ++t) {
         sc.t = t;
@@ -1491,9 +1497,12 @@ __global__ void __launch_bounds__(kThreads, 1) monokernel(const __grid_constant_
             ok = false;
             break;
         }
-        const __nv_bfloat16* erow = embed + (size_t)tok * dm.d;
-        for (int i = own0 + tid; i < own1; i += kConsumerThreads)
-            sm.xown[i - own0] = __bfloat162float(erow[i]);  // the residual rows this CTA updates in O and D
+        {
+            const __nv_bfloat16* erow = embed + (size_t)tok * dm.d;
+            const int own0 = sm.geom[kGeomOwn], own1 = sm.geom[kGeomOwn + 1];
+            for (int i = own0 + tid; i < own1; i += kConsumerThreads)
+                sm.xown[i - own0] = __bfloat162float(erow[i]);  // the residual rows this CTA updates in O and D
+        }
 
         // The step's phases in order: per layer QKV, ATT, O, GU, D, then the LM head if this
         // step's logits are needed. One loop with one call site per phase kind keeps the
@@ -1519,6 +1528,7 @@ __global__ void __launch_bounds__(kThreads, 1) monokernel(const __grid_constant_
                     ph == kQKV ? lb + P.lay.l_attn_norm : ph == kGU ? lb + P.lay.l_ffn_norm : P.arena + P.lay.final_norm);
                 const bool from_embed = ph == kQKV && l == 0;
                 const unsigned long long* xin = tagged + P.lay.x / 8 + (ph == kGU ? 0 : dm.d);  // O's or D's output
+                const __nv_bfloat16* erow = embed + (size_t)sm.flag[2] * dm.d;  // this step's token row
                 load_rmsnorm(sm, from_embed ? nullptr : xin, tag_in, from_embed ? erow : nullptr, gain, dm.d, dm.eps, P,
                              ctl, ok);
             }
@@ -1540,7 +1550,7 @@ __global__ void __launch_bounds__(kThreads, 1) monokernel(const __grid_constant_
             if (q + 1 < nphase) {
                 if (!(ok = phase_end(ok, tr))) break;
             } else {
-                if (!(ok = grid_sync(sm, epoch, base, P, ctl, ok, tr))) break;
+                if (!(ok = grid_sync(sm, P, ctl, ok, tr))) break;
             }
         }
     }
