@@ -56,6 +56,22 @@ def launch_traffic(bytes_launch: float):
     return cap["dram_bytes"] / cap["algorithmic_bytes"] * bytes_launch
 
 
+def max_over_ranks(values, device):
+    """Element-wise maximum of `values` over all ranks of the default process group (the
+    values themselves with one rank). Used for every time the benchmark reports."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t]
+
+
+def replica_throughput(tokens_per_rank: int, world: int, max_ms: float) -> float:
+    """Whole-job tokens/s of `world` independent replicas: all tokens over the slowest rank's time."""
+    return tokens_per_rank * world / (max_ms * 1e-3)
+
+
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -285,11 +301,9 @@ def main():
     total_ms = t0.elapsed_time(t1)
     kern_ms = [a.elapsed_time(b) for a, b in ev]
     launches = dec.info().launches - launches0
-    t = torch.tensor([total_ms, max(kern_ms)], dtype=torch.float64, device=dev)
+    total_ms, kern_max = max_over_ranks([total_ms, max(kern_ms)], dev)
     if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
         dist.barrier()
-    total_ms, kern_max = float(t[0]), float(t[1])
 
     # ---- end to end through the public host-memory call
     h_in = start.pin_memory()
@@ -305,10 +319,7 @@ def main():
         dec.generate(h_in, w.start_pos, w.n_gen, h_out)
     e1.record(stream)
     torch.cuda.synchronize(dev)
-    e2e_ms = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
-    e2e_ms = float(e2e_ms[0])
+    e2e_ms = max_over_ranks([e0.elapsed_time(e1)], dev)[0]
 
     # ---- roofline of the monokernel: algorithmic bytes per launch / launch time
     cfg = dec.cfg
@@ -320,8 +331,7 @@ def main():
 
     line = None
     if rank == 0:
-        tokens = args.steps * w.n_gen * world
-        value = tokens / (total_ms * 1e-3)
+        value = replica_throughput(args.steps * w.n_gen, world, total_ms)
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
@@ -336,7 +346,7 @@ def main():
                          "launch_ms": mean_kern_ms},
             "tokens_per_s_per_launch": w.n_gen / (mean_kern_ms * 1e-3),
             "roofline_tokens_per_s": w.n_gen / (bytes_launch / (peak * 1e9)),
-            "e2e": {"value": args.steps * w.n_gen * world / (e2e_ms * 1e-3), "unit": "tokens/s",
+            "e2e": {"value": replica_throughput(args.steps * w.n_gen, world, e2e_ms), "unit": "tokens/s",
                     "h2d_bytes_per_step": 4 * w.n_pending, "d2h_bytes_per_step": 4 * w.n_gen},
             "gpu_launches": launches, "launches_per_token": launches / (args.steps * w.n_gen),
             "clocks": clk.summary(),

@@ -141,6 +141,14 @@ int kd_decode(kd_ctx *ctx, int32_t n_gen, int32_t *d_tokens_out, float *d_logits
 int kd_generate(kd_ctx *ctx, const int32_t *h_tokens, int32_t n_tokens, int32_t kv_len,
                 int32_t n_gen, int32_t *h_tokens_out);
 
+/* Time limit, in nanoseconds (>= 1), of every device-side wait of later launches: a grid
+ * barrier, a weight stage, a tagged activation, a KV-row guard. The default is 1 s, or
+ * KD_TIMEOUT_MS milliseconds when that environment variable is set at kd_create. A wait that
+ * exceeds its limit sets the device status and every CTA stops (none traps, none hangs:
+ * copies already in flight are awaited under a separate fixed bound); kd_sync then returns
+ * KD_ETIMEOUT and the handle needs kd_reset. Returns KD_EINVAL for ns < 1. */
+int kd_set_timeout(kd_ctx *ctx, int64_t ns);
+
 /* Wait for the stream, then return the device status of the last decode (KD_OK,
  * KD_ETIMEOUT, KD_ETOKEN) or a CUDA error. */
 int kd_sync(kd_ctx *ctx);

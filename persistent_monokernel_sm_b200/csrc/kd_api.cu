@@ -484,6 +484,12 @@ int kd_set_trace(kd_ctx* c, unsigned long long* d_buf, int64_t n_words, int32_t 
     return KD_OK;
 }
 
+int kd_set_timeout(kd_ctx* c, int64_t ns) {
+    if (!c || ns < 1) return KD_EINVAL;
+    c->timeout_ns = ns;
+    return KD_OK;
+}
+
 int32_t kd_position(const kd_ctx* c) { return c ? c->pos : -1; }
 
 int kd_get_info(const kd_ctx* c, kd_info* info) {

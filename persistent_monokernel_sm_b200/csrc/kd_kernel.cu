@@ -1394,13 +1394,16 @@ struct Producer {
         // Let every copy already issued land before the CTA exits: when the consumers have
         // stopped early (a refused token, a wait that gave up) nobody else waits for them.
         // On a normal run these stages were consumed already and each test passes at once.
+        // The bound is fixed and generous, not the launch's wait limit (which may be tiny):
+        // an issued copy always completes within microseconds.
         {
+            constexpr uint64_t kDrainNs = 100000000ull;  // 100 ms
             const int first = k > P.ns ? k - P.ns : 0;
             for (int kk = first; kk < k; ++kk) {
                 const uint32_t a = smem_u32(&sm.full[kk % P.ns]);
                 const uint32_t par = (uint32_t)((kk / P.ns) & 1);
                 const uint64_t t0 = globaltimer();
-                while (!mbar_try_wait(a, par) && globaltimer() - t0 < (uint64_t)P.timeout_ns) {
+                while (!mbar_try_wait(a, par) && globaltimer() - t0 < kDrainNs) {
                 }
             }
         }

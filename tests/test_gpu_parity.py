@@ -185,6 +185,33 @@ def test_token_outside_vocab_stops_the_launch(kd):
     assert np.array_equal(again.cpu().numpy(), ref)
 
 
+def test_wait_limit_reports_timeout_and_recovers(kd):
+    """With a 1 ns wait limit the first wait that does not succeed at once gives up: the
+    launch stops without trapping or hanging, kd_sync reports KD_ETIMEOUT, decode is refused
+    until kd_reset, and with the normal limit back the handle decodes exactly as before."""
+    w = synth.get("tiny")
+    W = weights_for("tiny")
+    prompt = synth.make_prompt(w).numpy()
+    dec = make_decoder(kd, w, W)
+    dec.reset(prompt, 0)
+    ref, _ = dec.decode(16)
+    dec.sync()
+    ref = ref.cpu().numpy().copy()
+    kd.kd_set_timeout(dec.h, 1)
+    dec.reset(prompt, 0)
+    dec.decode(16)
+    with pytest.raises(kd.KdError) as e:
+        dec.sync()
+    assert e.value.code == -6
+    with pytest.raises(kd.KdError):
+        dec.decode(1)
+    kd.kd_set_timeout(dec.h, 1_000_000_000)
+    dec.reset(prompt, 0)
+    again, _ = dec.decode(16)
+    dec.sync()
+    assert np.array_equal(again.cpu().numpy(), ref)
+
+
 # ------------------------------------------------------------------ 0.5B: every step
 
 def test_half_billion_forced_and_greedy(kd):
