@@ -35,8 +35,8 @@ SPEC_HBM_GBS = 8000.0          # B200 HBM3e specification
 # (dram__bytes_read.sum + dram__bytes_write.sum of one launch decoding 8 tokens of the 2B model
 # at a 4k context; profiles/monokernel_2b-4k_8tok_counters.md). It holds for the kernel source
 # it was taken on only: when csrc/kd_kernel.cu no longer has this SHA-256, traffic is null.
-TRAFFIC_CAPTURE = {"kernel_sha256": "31353dcb370cf64ec235862dcb2ddd9e3454fcde39746b655278bb761bcc36d4",
-                   "dram_bytes": 32998681000.0 + 9641728.0, "algorithmic_bytes": 32998424576.0}
+TRAFFIC_CAPTURE = {"kernel_sha256": "1ce29b35780aaf3994a3ec3d2bbc969f2b70c587fbff10571c48e468f432e7d7",
+                   "dram_bytes": 32994343168.0 + 64696064.0, "algorithmic_bytes": 32998424576.0}
 FALLBACK_HBM_GBS = 6650.0       # earlier measurement on this machine, if no measured peaks file
 
 

@@ -302,8 +302,6 @@ struct Smem {
     int* flag;              // broadcast slots
     uint64_t* full;         // mbarriers
     uint64_t* empty;
-    float* sp;              // per-stage partial sums [slot][row][warp]
-    int* scnt;              // per-stage arrival counts [slot]
     float* xown;            // the residual rows this CTA owns (updated by O and D)
     __nv_bfloat16* kvcur;   // the current position's K and V row of the head being attended
     int* geom;              // this CTA's GEMV rows per phase and owned residual rows (cta_geometry)
@@ -313,7 +311,7 @@ struct Smem {
 // Byte offsets of the shared-memory regions; each starts on a 128-byte boundary (vector
 // loads and bulk-copy destinations need 16). Used by the kernel and for the launch size.
 struct SmemLayout {
-    size_t ring, xs, qs, rope, red, best, flag, full, empty, sp, scnt, xown, kvcur, geom, att, total;
+    size_t ring, xs, qs, rope, red, best, flag, full, empty, xown, kvcur, geom, att, total;
 };
 __host__ __device__ inline SmemLayout smem_layout(int ns, int xs_floats, int xown_floats) {
     SmemLayout L{};
@@ -332,8 +330,6 @@ __host__ __device__ inline SmemLayout smem_layout(int ns, int xs_floats, int xow
     L.flag = take(16 * 4);
     L.full = take((size_t)kMaxStages * 8);
     L.empty = take((size_t)kMaxStages * 8);
-    L.sp = take((size_t)kMaxStages * kMaxRows * 4);
-    L.scnt = take((size_t)kMaxStages * 4);
     L.xown = take((size_t)xown_floats * 4);
     L.kvcur = take(2 * 128 * 2);
     L.geom = take((size_t)kGeomWords * 4);
@@ -354,8 +350,6 @@ __device__ __forceinline__ Smem carve(const Params& P, uint8_t* base) {
     s.flag = reinterpret_cast<int*>(base + L.flag);
     s.full = reinterpret_cast<uint64_t*>(base + L.full);
     s.empty = reinterpret_cast<uint64_t*>(base + L.empty);
-    s.sp = reinterpret_cast<float*>(base + L.sp);
-    s.scnt = reinterpret_cast<int*>(base + L.scnt);
     s.xown = reinterpret_cast<float*>(base + L.xown);
     s.kvcur = reinterpret_cast<__nv_bfloat16*>(base + L.kvcur);
     s.geom = reinterpret_cast<int*>(base + L.geom);
@@ -550,6 +544,14 @@ __device__ __forceinline__ void load_rmsnorm(const Smem& sm, const unsigned long
                                              const Params& P, unsigned long long* ctl, bool& ok) {
     const int tid = threadIdx.x;
     constexpr int step = kConsumerThreads * 4;
+    // With K <= 2 * step (every model up to d_model 2048) each thread's gains are read here,
+    // before the input is polled, so the normalisation below waits on no global load.
+    const bool early = K <= 2 * step;
+    uint2 g0 = make_uint2(0u, 0u), g1 = make_uint2(0u, 0u);
+    if (early) {
+        if (tid * 4 < K) g0 = __ldg(reinterpret_cast<const uint2*>(gain + tid * 4));
+        if (tid * 4 + step < K) g1 = __ldg(reinterpret_cast<const uint2*>(gain + tid * 4 + step));
+    }
     float ss = 0.f;
     for (int k0 = tid * 4; k0 < K; k0 += 2 * step) {
         const int k1 = k0 + step;
@@ -581,9 +583,9 @@ __device__ __forceinline__ void load_rmsnorm(const Smem& sm, const unsigned long
 #pragma unroll
     for (int w = 0; w < kConsumerWarps; ++w) tot += sm.red[w];
     const float inv = 1.0f / sqrtf(tot / (float)K + eps);
-    for (int k = tid * 4; k < K; k += kConsumerThreads * 4) {
+    for (int k = tid * 4; k < K; k += step) {
         float4* p = reinterpret_cast<float4*>(&sm.xs[xs_index(k, K)]);
-        const uint2 gw = __ldg(reinterpret_cast<const uint2*>(gain + k));
+        const uint2 gw = early ? (k == tid * 4 ? g0 : g1) : __ldg(reinterpret_cast<const uint2*>(gain + k));
         float4 v = *p;
         v.x = (v.x * inv) * bf_lo(gw.x);
         v.y = (v.y * inv) * bf_hi(gw.x);
@@ -822,18 +824,15 @@ __device__ __forceinline__ void run_gemv(const Params& P, const Smem& sm, unsign
     }
 }
 
-// Loads that read either the shared-memory ring or, for the current position, the cache
-// itself (written during this launch: L2 only).
-__device__ __forceinline__ uint4 ld16(const __nv_bfloat16* p, bool global) {
-    return global ? __ldcg(reinterpret_cast<const uint4*>(p)) : *reinterpret_cast<const uint4*>(p);
-}
+// Loads of K and V rows from a stage of the shared-memory ring.
+__device__ __forceinline__ uint4 ld16(const __nv_bfloat16* p) { return *reinterpret_cast<const uint4*>(p); }
 template <int E>
-__device__ __forceinline__ void ld_v(const __nv_bfloat16* p, bool global, float (&v)[E]) {
+__device__ __forceinline__ void ld_v(const __nv_bfloat16* p, float (&v)[E]) {
     if constexpr (E == 4) {
-        const uint2 w = global ? __ldcg(reinterpret_cast<const uint2*>(p)) : *reinterpret_cast<const uint2*>(p);
+        const uint2 w = *reinterpret_cast<const uint2*>(p);
         v[0] = bf_lo(w.x), v[1] = bf_hi(w.x), v[2] = bf_lo(w.y), v[3] = bf_hi(w.y);
     } else {
-        const uint32_t w = global ? __ldcg(reinterpret_cast<const unsigned int*>(p)) : *reinterpret_cast<const uint32_t*>(p);
+        const uint32_t w = *reinterpret_cast<const uint32_t*>(p);
         v[0] = bf_lo(w), v[1] = bf_hi(w);
     }
 }
@@ -966,7 +965,7 @@ __device__ __forceinline__ void run_attention(const Params& P, const Smem& sm_re
     // kb / vb): lanes 4j..4j+3 score position j of both blocks, then all lanes fold the up
     // to 16 V rows into their output dims with a single rescale.
     auto pass2 = [&](const __nv_bfloat16* ka, const __nv_bfloat16* va, int na, const __nv_bfloat16* kb,
-                     const __nv_bfloat16* vb, int nb, bool global) {
+                     const __nv_bfloat16* vb, int nb) {
         const bool ma = pj < na, mb = pj < nb;
         float sa[GMAX][2], sb[GMAX][2];
 #pragma unroll
@@ -974,8 +973,8 @@ __device__ __forceinline__ void run_attention(const Params& P, const Smem& sm_re
 #pragma unroll
         for (int i = 0; i < CPL; ++i) {
             const int c = qq + 4 * i;
-            const uint4 wa = ma ? ld16(ka + (size_t)pj * HD + c * 8, global) : make_uint4(0, 0, 0, 0);
-            const uint4 wb = mb ? ld16(kb + (size_t)pj * HD + c * 8, global) : make_uint4(0, 0, 0, 0);
+            const uint4 wa = ma ? ld16(ka + (size_t)pj * HD + c * 8) : make_uint4(0, 0, 0, 0);
+            const uint4 wb = mb ? ld16(kb + (size_t)pj * HD + c * 8) : make_uint4(0, 0, 0, 0);
 #pragma unroll
             for (int h = 0; h < GMAX; ++h) {
                 if (h < r) {
@@ -1029,8 +1028,8 @@ __device__ __forceinline__ void run_attention(const Params& P, const Smem& sm_re
 #pragma unroll
         for (int jj = 0; jj < 8; ++jj) {
             float v0[E], v1[E];
-            if (jj < na) ld_v<E>(va + (size_t)jj * HD + lane * E, global, v0);
-            if (jj < nb) ld_v<E>(vb + (size_t)jj * HD + lane * E, global, v1);
+            if (jj < na) ld_v<E>(va + (size_t)jj * HD + lane * E, v0);
+            if (jj < nb) ld_v<E>(vb + (size_t)jj * HD + lane * E, v1);
 #pragma unroll
             for (int h = 0; h < GMAX; ++h) {
                 if (h < r) {
@@ -1084,7 +1083,7 @@ __device__ __forceinline__ void run_attention(const Params& P, const Smem& sm_re
                 if (na == 0 && nb > 0) {  // pass2 wants a non-empty first block
                     ka = kb, va = vb, na = nb, nb = 0;
                 }
-                if (na > 0) pass2(ka, va, na, kb, vb, nb, false);
+                if (na > 0) pass2(ka, va, na, kb, vb, nb);
                 __syncwarp();
                 if (lane == kSyncLane) {
                     mbar_arrive(smem_u32(&sm.empty[ra.slot]));
@@ -1382,9 +1381,11 @@ struct Producer {
         ld.geom = pf.geom = sm.geom;
         ld.begin(P);
         pf.begin(P);
+        // The L2 lookahead (off unless requested) runs a second cursor P.prefetch stages ahead.
+        const bool lookahead = P.prefetch > 0;
         for (int i = 0; i < P.prefetch && !pf.done; ++i, pf.next(P)) prefetch(pf);
         while (ok && !ld.done) {
-            if (!pf.done) {
+            if (lookahead && !pf.done) {
                 prefetch(pf);
                 pf.next(P);
             }
@@ -1431,7 +1432,6 @@ __global__ void __launch_bounds__(kThreads, 1) monokernel(const __grid_constant_
         for (int s = 0; s < P.ns; ++s) {
             mbar_init(smem_u32(&sm.full[s]), 1);
             mbar_init(smem_u32(&sm.empty[s]), kGroupWarps);  // every warp of the slot's group releases
-            sm.scnt[s] = 0;
         }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         cta_geometry(P, blockIdx.x, sm.geom);
