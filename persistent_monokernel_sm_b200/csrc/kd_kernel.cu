@@ -725,47 +725,65 @@ __device__ __forceinline__ void run_gemv_t(const Params& P, const Smem& sm_ref, 
         return (a0 + a1) + (a2 + a3);
     };
 
-    // Stages are taken two at a time: the four dot products (two rows of each stage) and their
-    // reductions interleave, and the per-stage bookkeeping is paid once per pair.
-    auto put = [&](int j, int n, float pa, float pb) {
-        if (rowa < n) pp[(j * g.R + rowa) * KS + ks] = pa;
-        if (dual && rowb < n) pp[(j * g.R + rowb) * KS + ks] = pb;
+    // Stages are taken four at a time, as two pairs. For each pair the four dot products (two
+    // rows of each stage) are formed and both slots handed back; the eight lane partials of
+    // the four stages are then reduced together. Three exchange levels (offsets 16, 8, 4) halve
+    // the values a lane holds at each step, so 4 + 2 + 1 shuffles leave each lane one value
+    // summed over 8 lanes; two plain levels (offsets 2, 1) complete the 32-lane sum. Value i
+    // (stage j + i / 2, row a for even i, row b for odd i) ends in lanes 4i..4i+3.
+    auto put = [&](int jj, int row, float z) {
+        if (jj < nst && row < min(g.R, g.row1 - (g.row0 + jj * g.R))) pp[(jj * g.R + row) * KS + ks] = z;
     };
-    for (int j = 0; j < nst; j += 2) {
-        const Ring ra = rg;
-        rg.advance(ns);
-        const bool two = j + 1 < nst;
-        const Ring rb = rg;
-        if (two) rg.advance(ns);
-        if (!ok) continue;
-        if (!wait_full(sm, ra, P, ctl, waited) || (two && !wait_full(sm, rb, P, ctl, waited))) {
-            ok = false;
-            continue;
-        }
-        if (threadIdx.x == 0 && j == 0) tr.mark(4);  // first stage of the phase ready
-        const int na = min(g.R, g.row1 - (g.row0 + j * g.R));            // rows in stage j
-        const int nb = two ? min(g.R, g.row1 - (g.row0 + (j + 1) * g.R)) : 0;  // rows in stage j + 1
-        const uint8_t* sa = sm.ring + (size_t)ra.slot * kStageBytes;
-        const uint8_t* sb = sm.ring + (size_t)rb.slot * kStageBytes;
-        float p0 = rowa < na ? dot_row(sa + rowa * rowbytes) : 0.f;
-        float p1 = dual && rowb < na ? dot_row(sa + rowb * rowbytes) : 0.f;
-        float p2 = rowa < nb ? dot_row(sb + rowa * rowbytes) : 0.f;
-        float p3 = dual && rowb < nb ? dot_row(sb + rowb * rowbytes) : 0.f;
+    for (int j = 0; j < nst; j += 4) {
+        float v[8];
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            p0 += __shfl_xor_sync(0xffffffffu, p0, o);
-            p1 += __shfl_xor_sync(0xffffffffu, p1, o);
-            p2 += __shfl_xor_sync(0xffffffffu, p2, o);
-            p3 += __shfl_xor_sync(0xffffffffu, p3, o);
+        for (int h = 0; h < 2; ++h) {  // stages j + 2h and j + 2h + 1
+            const int jj = j + 2 * h;
+            float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;
+            if (jj < nst) {
+                const Ring ra = rg;
+                rg.advance(ns);
+                const bool two = jj + 1 < nst;
+                const Ring rb = rg;
+                if (two) rg.advance(ns);
+                if (ok) {
+                    if (!wait_full(sm, ra, P, ctl, waited) || (two && !wait_full(sm, rb, P, ctl, waited))) {
+                        ok = false;
+                    } else {
+                        if (threadIdx.x == 0 && jj == 0) tr.mark(4);  // first stage of the phase ready
+                        const int na = min(g.R, g.row1 - (g.row0 + jj * g.R));                   // rows in stage jj
+                        const int nb = two ? min(g.R, g.row1 - (g.row0 + (jj + 1) * g.R)) : 0;  // and in jj + 1
+                        const uint8_t* sa = sm.ring + (size_t)ra.slot * kStageBytes;
+                        const uint8_t* sb = sm.ring + (size_t)rb.slot * kStageBytes;
+                        p0 = rowa < na ? dot_row(sa + rowa * rowbytes) : 0.f;
+                        p1 = dual && rowb < na ? dot_row(sa + rowb * rowbytes) : 0.f;
+                        p2 = rowa < nb ? dot_row(sb + rowa * rowbytes) : 0.f;
+                        p3 = dual && rowb < nb ? dot_row(sb + rowb * rowbytes) : 0.f;
+                        __syncwarp();
+                        if (lane == kSyncLane) {  // done with the stages
+                            mbar_arrive(smem_u32(&sm.empty[ra.slot]));
+                            if (two) mbar_arrive(smem_u32(&sm.empty[rb.slot]));
+                        }
+                    }
+                }
+            }
+            v[4 * h] = p0, v[4 * h + 1] = p1, v[4 * h + 2] = p2, v[4 * h + 3] = p3;
         }
-        __syncwarp();
-        if (lane == kSyncLane) {  // done with the stages
-            mbar_arrive(smem_u32(&sm.empty[ra.slot]));
-            if (two) mbar_arrive(smem_u32(&sm.empty[rb.slot]));
-        }
-        if (lane == 0) {
-            put(j, na, p0, p1);
-            if (two) put(j + 1, nb, p2, p3);
+        const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4;
+        float w4[4], w2[2];
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+            w4[k] = (b4 ? v[4 + k] : v[k]) + __shfl_xor_sync(0xffffffffu, b4 ? v[k] : v[4 + k], 16);
+#pragma unroll
+        for (int k = 0; k < 2; ++k)
+            w2[k] = (b3 ? w4[2 + k] : w4[k]) + __shfl_xor_sync(0xffffffffu, b3 ? w4[k] : w4[2 + k], 8);
+        float z = (b2 ? w2[1] : w2[0]) + __shfl_xor_sync(0xffffffffu, b2 ? w2[0] : w2[1], 4);
+        z += __shfl_xor_sync(0xffffffffu, z, 2);
+        z += __shfl_xor_sync(0xffffffffu, z, 1);
+        if ((lane & 3) == 0 && ok) {
+            const int i = lane >> 2;  // value index: 4 * b4 + 2 * b3 + b2
+            if ((i & 1) == 0) put(j + (i >> 1), rowa, z);
+            else if (dual) put(j + (i >> 1), rowb, z);
         }
     }
     if (threadIdx.x == 0) tr.mark(5);  // this warp's stages done
