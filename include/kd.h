@@ -61,9 +61,10 @@ enum {
 };
 
 /* Model shape. Limits: n_layers >= 1; head_dim in {64, 128}; n_heads a multiple of
- * n_kv_heads with n_heads / n_kv_heads <= 8; n_kv_heads <= 16; d_model, ffn_dim multiples
- * of 64 with 2*d_model*2 <= 32768 and ffn_dim*2 <= 32768 (one row pair / one row fits a
- * 32 KB pipeline stage); vocab >= 1; max_seq >= 1 (KV positions held). */
+ * n_kv_heads with n_heads / n_kv_heads <= 8; n_kv_heads <= 16; d_model a multiple of 256
+ * between 256 and 8192 whose slices of at most 1024 elements are multiples of 256 (every
+ * GEMV row is streamed as whole 16-byte chunks per lane: 256, 512, ..., 4096, 6144, 8192
+ * qualify; 5120 does not); ffn_dim >= 1; vocab >= 1; max_seq >= 1 (KV positions held). */
 typedef struct kd_config {
     int32_t n_layers, d_model, n_heads, n_kv_heads, head_dim, ffn_dim, vocab, max_seq;
     float rms_eps, rope_theta;
@@ -88,11 +89,15 @@ typedef struct kd_info {
     int32_t smem_bytes;    /* dynamic shared memory per CTA */
     int32_t stages;        /* weight/KV pipeline stages per CTA */
     int32_t stage_bytes;   /* bytes per stage */
-    int32_t attn_pieces;   /* CTAs per kv head in the split-K attention phase */
+    int32_t attn_pieces;   /* CTAs per kv head: attention pieces, and the shares of that kv
+                              head's Q/K/V rows and output-projection inputs */
     int64_t arena_bytes;   /* bytes of the arena layout */
     int64_t weight_bytes;  /* bytes of the weights inside the arena */
     int64_t kv_bytes;      /* bytes of the KV cache inside the arena */
     int64_t launches;      /* kernel launches made through this handle so far */
+    int64_t ctl_offset;    /* byte offset of the control words in the arena (word 0: the
+                              monotonic 64-bit count of cross-CTA sync arrivals); exposed for
+                              diagnostics and tests, not to be written while a decode runs */
 } kd_info;
 
 typedef struct kd_ctx kd_ctx;
@@ -141,8 +146,8 @@ int kd_decode(kd_ctx *ctx, int32_t n_gen, int32_t *d_tokens_out, float *d_logits
 int kd_generate(kd_ctx *ctx, const int32_t *h_tokens, int32_t n_tokens, int32_t kv_len,
                 int32_t n_gen, int32_t *h_tokens_out);
 
-/* Time limit, in nanoseconds (>= 1), of every device-side wait of later launches: a grid
- * barrier, a weight stage, a tagged activation, a KV-row guard. The default is 1 s, or
+/* Time limit, in nanoseconds (>= 1), of every device-side wait of later launches: a
+ * cross-CTA sync, a weight stage, a tagged activation, a KV-row guard. The default is 1 s, or
  * KD_TIMEOUT_MS milliseconds when that environment variable is set at kd_create. A wait that
  * exceeds its limit sets the device status and every CTA stops (none traps, none hangs:
  * copies already in flight are awaited under a separate fixed bound); kd_sync then returns
@@ -159,13 +164,14 @@ int kd_sync(kd_ctx *ctx);
  * a host that can only lend the library buffers it registered in advance).
  * It resets the request like kd_reset (d_tokens: device int32 [n_tokens], the first at
  * position kv_len) and generates n_gen tokens in one launch, exactly like kd_decode, but the
- * activation vectors, attention partials, control words and pending tokens live in a 1 MiB
- * array inside the library (loaded on every GPU that loads libkd, held until exit) instead of
- * in the arena's scratch region. The weights and KV cache are still the handle's arena.
- * Inputs and outputs as for kd_decode; calls KD_EINVAL with a message when this model and
- * n_tokens need more than the 1 MiB. It calls no allocator: the control words are cleared
- * with a memset and the tokens copied in, then it waits for the launch and returns its
- * device status. The array keeps the last call's contents and every call shares it, so
+ * split-K sums, the tagged Q/K/V words and attention records, the control words and the
+ * pending tokens live in a 1 MiB array inside the library (loaded on every GPU that loads
+ * libkd, held until exit) instead of in the arena's scratch region. The weights and the KV
+ * cache are still the handle's arena: the call appends to that cache at positions
+ * [kv_len, kv_len + steps) like kd_decode would. Inputs and outputs as for kd_decode; returns
+ * KD_EINVAL with a message when this model and n_tokens need more than the 1 MiB. It calls no
+ * allocator: the scratch it uses is cleared with a memset and the tokens copied in, then it
+ * waits for the launch and returns its device status. The array keeps the last call's contents and every call shares it, so
  * calls that overlap on the GPU (two streams, two handles) race: serialise them. The first
  * call on a device looks the array's address up (cudaGetSymbolAddress), so make that first
  * call outside any stream capture. The handle's position and pending tokens are not changed. */
@@ -173,14 +179,16 @@ int kd_decode_noalloc(kd_ctx *ctx, const int32_t *d_tokens, int32_t n_tokens, in
                       int32_t n_gen, int32_t *d_tokens_out, float *d_logits_out);
 
 /* Optional phase trace for performance analysis (off by default). While set, every
- * decode launch has each CTA with index % every == 0 record, per phase and in phase order,
- * a row of eight SM-clock stamps: phase begin, activation vector loaded, arrival at the grid
- * barrier, barrier passed, then (attention phase only, else 0) q loaded, cache pieces done,
- * partial record written, cross-CTA combine done. Traced CTA i owns rows [i * R, (i + 1) * R)
- * of the buffer, where R = n_words / (8 * ceil(grid / every)); its last row holds the producer
- * warp's cycles blocked on a free pipeline stage, cycles blocked on a KV epoch, stages issued
- * and total cycles. d_buf: device memory of n_words uint64 (caller-owned); NULL turns
- * tracing off. */
+ * decode launch has each CTA with index % every == 0 record, per phase (Q/K/V, attention,
+ * output projection, gate/up, down, LM head) and in phase order, a row of eight words:
+ * the phase id (step << 16 | layer << 4 | phase 0..5), then SM-clock stamps of phase begin,
+ * inputs ready (the cross-CTA sync passed or the tagged inputs polled), compute done and
+ * phase end, then the cycles spent waiting for weight / KV stages, then two zero words.
+ * Traced CTA i owns rows [i * R, (i + 1) * R) of the buffer, where
+ * R = n_words / (8 * ceil(grid / every)); its last row holds the producer warp's cycles
+ * blocked on a free pipeline stage, cycles blocked on KV rows written during the launch,
+ * stages issued and total cycles. d_buf: device memory of n_words uint64 (caller-owned);
+ * NULL turns tracing off. */
 int kd_set_trace(kd_ctx *ctx, unsigned long long *d_buf, int64_t n_words, int32_t every);
 
 /* Next KV position to be written (host-side view, valid once calls were enqueued). */

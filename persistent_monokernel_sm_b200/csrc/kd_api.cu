@@ -15,7 +15,7 @@ using namespace kd;
 
 namespace {
 
-constexpr int kMaxGrid = 256;  // partial-record room for up to this many CTAs
+constexpr int kMaxGrid = 256;  // attention-record room for up to this many CTAs
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
@@ -25,10 +25,9 @@ bool valid_config(const kd_config* c) {
     if (c->head_dim != 64 && c->head_dim != 128) return false;
     if (c->n_heads % c->n_kv_heads || c->n_heads / c->n_kv_heads > kMaxGroup) return false;
     if (c->n_kv_heads > kMaxKvHeads) return false;
-    if (c->d_model % 64 || c->ffn_dim <= 0 || c->ffn_dim % 64) return false;
-    if (4LL * c->d_model > kStageBytes || 2LL * c->ffn_dim > kStageBytes) return false;
-    if (2LL * c->n_heads * c->head_dim > kStageBytes) return false;
-    if (c->vocab < 1 || c->max_seq < 1) return false;
+    Shape sh;
+    if (!make_shape(c->d_model, &sh)) return false;
+    if (c->ffn_dim <= 0 || c->vocab < 1 || c->max_seq < 1) return false;
     if (!(c->rms_eps >= 0.f) || !(c->rope_theta > 0.f)) return false;
     return true;
 }
@@ -64,9 +63,9 @@ Layout make_layout(const Dims& d) {
     y.l_attn_norm = ltake(D * 2);
     y.l_ffn_norm = ltake(D * 2);
     y.l_wqkv = ltake((size_t)d.qkv_rows * D * 2);
-    y.l_wo = ltake(D * d.qd * 2);
+    y.l_wot = ltake((size_t)d.qd * D * 2);
     y.l_wgu = ltake((size_t)2 * d.F * D * 2);
-    y.l_wd = ltake(D * d.F * 2);
+    y.l_wdt = ltake((size_t)d.F * D * 2);
     y.layer_stride = lo;
     off = y.layer0 + (size_t)d.L * y.layer_stride;
     y.weights_end = off;
@@ -75,11 +74,9 @@ Layout make_layout(const Dims& d) {
     y.kcache = take(kv);
     y.vcache = take(kv);
     y.kv_bytes = 2 * kv;
-    y.x = take(2 * D * 8);                 // tagged: residual after O, after D
-    y.qkv = take((size_t)d.qkv_rows * 8);  // tagged raw q/k/v projections (repacked row order)
-    y.o = take((size_t)d.qd * 8);          // tagged attention output
-    y.gu = take((size_t)d.F * 8);          // tagged FFN hidden vector silu(gate) * up
-    y.part = take((size_t)kMaxGrid * d.r * (d.hd + 2) * 4);
+    y.delta = take((size_t)3 * D * 4);                             // split-K sums, 3 rotating buffers
+    y.qkv = take((size_t)d.qkv_rows * 8);                          // tagged q / k / v of the step
+    y.rec = take((size_t)kMaxGrid * d.r * (d.hd + 2) * 8);         // tagged attention records
     y.ctl = take((size_t)kCtlWords * 8);
     y.tokens_in = take((size_t)d.S * 4);
     y.tokens_out = take((size_t)d.S * 4);  // staging for kd_generate
@@ -93,16 +90,16 @@ struct kd_ctx {
     kd_config cfg;
     Dims dm;
     Layout lay;
+    Shape sh;
     uint8_t* arena;
     cudaStream_t stream;
     int device;
-    int nb, smem, ns, pieces, pos_per_stage, xs_floats, xown_floats;
+    int nb, smem, ns, pieces, blk, work_floats, hin_floats;
     bool has_weights, failed;
     int pos, n_pending;
     long long launches;
     long long timeout_ns;
-    int prefetch, inflight;
-    uint32_t tag;  // tag base of the next launch (advanced by the phases each launch runs)
+    uint32_t tag;  // tag base of the next launch (advanced by the tagged phases each launch runs)
     unsigned long long* trace;
     int trace_every, trace_rows;
     char err[512];
@@ -129,25 +126,22 @@ static int fail(kd_ctx* c, int code, const char* fmt, ...) {
 
 namespace {
 
-// dst row r of the fused [q; k; v] projection: q and k heads hold RoPE pairs (i, i + hd/2)
-// in adjacent rows (2i, 2i + 1); v rows keep their order.
+// Row r of the kv-head-major [q; k; v] projection of one layer. Kv head g owns rows
+// [g * (r + 2) * hd, (g + 1) * (r + 2) * hd): its r q heads, its k head, its v head. q and k
+// heads hold RoPE pairs (i, i + hd/2) in adjacent rows (2i, 2i + 1); v rows keep their order.
 __global__ void repack_qkv(uint8_t* dst_layer0, size_t layer_stride, size_t off, const uint16_t* wq,
                            const uint16_t* wk, const uint16_t* wv, Dims dm) {
-    const int r = blockIdx.x, l = blockIdx.y;
+    const int row = blockIdx.x, l = blockIdx.y;
+    const int per = (dm.r + 2) * dm.hd;
+    const int g = row / per, rr = row % per;
+    const int seg = rr / dm.hd, j = rr % dm.hd;
+    const int pj = (j >> 1) + ((j & 1) ? dm.hd / 2 : 0);  // RoPE-pair order
     const uint16_t* src;
-    int row;
-    if (r < dm.qd + dm.kvd) {
-        const bool isq = r < dm.qd;
-        const int rr = isq ? r : r - dm.qd;
-        const int h = rr / dm.hd, j = rr % dm.hd;
-        row = h * dm.hd + (j >> 1) + ((j & 1) ? dm.hd / 2 : 0);
-        src = isq ? wq + (size_t)l * dm.qd * dm.d : wk + (size_t)l * dm.kvd * dm.d;
-    } else {
-        row = r - dm.qd - dm.kvd;
-        src = wv + (size_t)l * dm.kvd * dm.d;
-    }
-    const uint4* s = reinterpret_cast<const uint4*>(src + (size_t)row * dm.d);
-    uint4* d = reinterpret_cast<uint4*>(dst_layer0 + (size_t)l * layer_stride + off + (size_t)r * dm.d * 2);
+    if (seg < dm.r) src = wq + ((size_t)l * dm.qd + (size_t)(g * dm.r + seg) * dm.hd + pj) * dm.d;
+    else if (seg == dm.r) src = wk + ((size_t)l * dm.kvd + (size_t)g * dm.hd + pj) * dm.d;
+    else src = wv + ((size_t)l * dm.kvd + (size_t)g * dm.hd + j) * dm.d;
+    const uint4* s = reinterpret_cast<const uint4*>(src);
+    uint4* d = reinterpret_cast<uint4*>(dst_layer0 + (size_t)l * layer_stride + off + (size_t)row * dm.d * 2);
     for (int i = threadIdx.x; i < dm.d / 8; i += blockDim.x) d[i] = s[i];
 }
 
@@ -161,7 +155,52 @@ __global__ void repack_gu(uint8_t* dst_layer0, size_t layer_stride, size_t off, 
     for (int i = threadIdx.x; i < dm.d / 8; i += blockDim.x) d[i] = s[i];
 }
 
+// dst [cols][rows] = src [rows][cols]^T for every layer (bf16), 32 x 32 tiles. Used for the
+// output projection ([d][Hq*hd] -> [Hq*hd][d]) and the down projection ([d][F] -> [F][d]),
+// so that a CTA's split-K share of either is one contiguous run of rows.
+__global__ void transpose_bf16(uint8_t* dst_layer0, size_t layer_stride, size_t off, const uint16_t* src, int rows,
+                               int cols) {
+    __shared__ uint16_t tile[32][33];
+    const int l = blockIdx.z;
+    const int c0 = blockIdx.x * 32, r0 = blockIdx.y * 32;
+    const uint16_t* s = src + (size_t)l * rows * cols;
+    uint16_t* d = reinterpret_cast<uint16_t*>(dst_layer0 + (size_t)l * layer_stride + off);
+    for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+        const int r = r0 + i, c = c0 + threadIdx.x;
+        if (r < rows && c < cols) tile[i][threadIdx.x] = s[(size_t)r * cols + c];
+    }
+    __syncthreads();
+    for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+        const int c = c0 + i, r = r0 + threadIdx.x;
+        if (r < rows && c < cols) d[(size_t)c * rows + r] = tile[threadIdx.x][i];
+    }
+}
+
 bool aligned16(const void* p) { return ((uintptr_t)p & 15) == 0; }
+
+// Shared-memory scratch (floats) of one CTA, sized for the largest user:
+//  hin:  the CTA's hidden values (down-projection inputs) or attention output dims;
+//  work: row-GEMV partials (rows x slices) of the Q/K/V, gate/up and LM-head shares, the
+//        attention scores and reductions of one softmax block, the split-K group sums, and
+//        the attention records the output projection gathers.
+void scratch_sizes(const Dims& d, const Shape& sh, int nb, int pieces, int blk, int* hin, int* work) {
+    const int units = (d.F + nb - 1) / nb + 1;
+    const int cols = d.r * d.hd / pieces + 2;
+    *hin = ((units > cols ? units : cols) + 31) & ~31;
+    const int gm = d.r <= 2 ? 2 : d.r <= 4 ? 4 : 8;
+    long long w = 0;
+    auto need = [&](long long v) { if (v > w) w = v; };
+    const int pairs = (d.r + 2) * d.hd / 2;
+    need((long long)2 * ((pairs + pieces - 1) / pieces) * sh.gs);  // Q/K/V rows
+    need((long long)2 * units * sh.gs);                             // gate/up rows
+    need((long long)((d.V + nb - 1) / nb) * sh.gs);                 // LM-head rows
+    const int pps = kStageBytes / (2 * d.hd), nq = d.hd / 32, npg = kConsumerThreads / (d.hd / 2);
+    const long long spart = 2LL * nq * gm * pps, vred = (long long)npg * gm * d.hd;
+    need((long long)(blk + 1) * gm + (spart > vred ? spart : vred));  // attention
+    if (sh.ug > 1) need((long long)sh.ug * d.d);                    // split-K group sums
+    need((long long)pieces * (4 + cols));                           // gathered attention records
+    *work = (int)((w + 31) & ~31LL);
+}
 
 }  // namespace
 
@@ -171,14 +210,12 @@ int kd_internal_view(kd_ctx* c, kd_ctx_view* v) {
     if (!c || !v) return KD_EINVAL;
     v->dm = &c->dm;
     v->lay = &c->lay;
+    v->sh = &c->sh;
     v->arena = c->arena;
     v->stream = c->stream;
     v->device = c->device, v->nb = c->nb, v->smem = c->smem, v->ns = c->ns;
-    v->pieces = c->pieces, v->pos_per_stage = c->pos_per_stage, v->xs_floats = c->xs_floats;
-    v->xown_floats = c->xown_floats;
+    v->pieces = c->pieces, v->blk = c->blk, v->work_floats = c->work_floats, v->hin_floats = c->hin_floats;
     v->timeout_ns = c->timeout_ns;
-    v->prefetch = c->prefetch;
-    v->inflight = c->inflight;
     v->has_weights = c->has_weights;
     return KD_OK;
 }
@@ -186,6 +223,21 @@ int kd_internal_view(kd_ctx* c, kd_ctx_view* v) {
 int kd_internal_fail(kd_ctx* c, int code, const char* msg) { return fail(c, code, "%s", msg); }
 
 void kd_internal_count_launch(kd_ctx* c) { c->launches += 1; }
+
+namespace kd {
+// The launch parameters that depend only on the handle (shared with kd_decode_noalloc).
+void fill_launch_shape(const kd_ctx_view& v, Params& p) {
+    p.dm = *v.dm;
+    p.sh = *v.sh;
+    p.nb = v.nb;
+    p.ns = v.ns;
+    p.pieces = v.pieces;
+    p.blk = v.blk;
+    p.work_floats = v.work_floats;
+    p.hin_floats = v.hin_floats;
+    p.timeout_ns = v.timeout_ns;
+}
+}  // namespace kd
 
 // ------------------------------------------------------------------ C ABI
 
@@ -217,14 +269,11 @@ int kd_create(const kd_config* cfg, void* d_arena, size_t arena_bytes, void* str
     c->cfg = *cfg;
     c->dm = make_dims(cfg);
     c->lay = make_layout(c->dm);
+    make_shape(c->dm.d, &c->sh);
     c->arena = (uint8_t*)d_arena;
     c->stream = (cudaStream_t)stream;
     c->timeout_ns = 1000000000LL;
     if (const char* t = getenv("KD_TIMEOUT_MS")) c->timeout_ns = atoll(t) * 1000000LL;
-    c->prefetch = 0;
-    if (const char* t = getenv("KD_PREFETCH")) c->prefetch = atoi(t);
-    c->inflight = 2;
-    if (const char* t = getenv("KD_INFLIGHT")) c->inflight = atoi(t);
     int rc = KD_OK;
     if (arena_bytes < c->lay.total || ((uintptr_t)d_arena & 255)) {
         rc = fail(c, KD_ENOMEM, "arena of %zu bytes at %p; need %zu bytes, 256-byte aligned", arena_bytes,
@@ -242,36 +291,30 @@ int kd_create(const kd_config* cfg, void* d_arena, size_t arena_bytes, void* str
         c->nb = prop.multiProcessorCount;
         if (c->nb > kMaxGrid) c->nb = kMaxGrid;
         c->pieces = c->nb / d.Hkv;
-        // attention stages: 8 positions per warp of a group (16 for hd 64), K then V rows
-        c->pos_per_stage = (d.hd == 128 ? 8 : 16) * kGroupWarps;
-        int xs = d.d;
-        if (d.qd > xs) xs = d.qd;
-        if (d.F > xs) xs = d.F;
-        const int merge = (kConsumerWarps + 1) * d.r * (d.hd + 2);  // warps' records + the current position's
-        if (merge > xs) xs = merge;
-        // every GEMV phase keeps its [row][slice] sums in xs until the phase ends
-        {
-            const int K[5] = {d.d, d.qd, d.d, d.F, d.d};
-            const long long units[5] = {d.qkv_rows / 2, d.d, d.F, d.d, d.V};
-            const int rpu[5] = {2, 1, 2, 1, 1};
-            for (int i = 0; i < 5; ++i) {
-                const int R = rows_per_stage(K[i], false);
-                const int slices = R >= 2 ? 16 / R : 8;
-                const long long rows = (units[i] + c->nb - 1) / c->nb * rpu[i];
-                if (rows * slices > xs) xs = (int)(rows * slices);
+        if (c->pieces < 1) rc = fail(c, KD_EINVAL, "%d CTAs cannot serve %d kv heads", c->nb, d.Hkv);
+    }
+    if (rc == KD_OK) {
+        // The ring takes what the scratch leaves: the largest softmax block (a multiple of a
+        // stage's positions, at most 1024) that still leaves room for 4 stages, then as many
+        // stages as fit (at most kMaxStages).
+        const Dims& d = c->dm;
+        const int pps = kStageBytes / (2 * d.hd);
+        Params p{};
+        p.dm = d;
+        c->ns = 0;
+        for (int blk = 1024; blk >= pps && c->ns == 0; blk -= pps) {
+            scratch_sizes(d, c->sh, c->nb, c->pieces, blk, &c->hin_floats, &c->work_floats);
+            p.hin_floats = c->hin_floats;
+            p.work_floats = c->work_floats;
+            p.ns = 0;
+            const int fixed = monokernel_smem_bytes(p);
+            const int ns = (kSmemLimit - fixed) / kStageBytes;
+            if (ns >= 4) {
+                c->ns = ns > kMaxStages ? kMaxStages : ns;
+                c->blk = blk;
             }
         }
-        c->xs_floats = (xs + 31) & ~31;
-        c->xown_floats = (d.d + c->nb - 1) / c->nb + 1;
-        Params p{};
-        p.xs_floats = c->xs_floats;
-        p.xown_floats = c->xown_floats;
-        p.ns = 1;
-        const int fixed = monokernel_smem_bytes(p) - kStageBytes;
-        c->ns = (kSmemLimit - fixed) / kStageBytes;
-        if (c->ns > kMaxStages) c->ns = kMaxStages;
-        c->ns -= c->ns % kGroups;  // consumer group g owns the slots g mod kGroups
-        if (c->ns < 2) rc = fail(c, KD_EINVAL, "activation buffers leave no room for a pipeline");
+        if (c->ns == 0) rc = fail(c, KD_EINVAL, "shared-memory scratch leaves no room for a pipeline");
         if (rc == KD_OK) {
             p.ns = c->ns;
             c->smem = monokernel_smem_bytes(p);
@@ -283,10 +326,10 @@ int kd_create(const kd_config* cfg, void* d_arena, size_t arena_bytes, void* str
         }
     }
     if (rc == KD_OK) {
-        // control words and the tagged activation buffers start at zero: tag 0 is never
-        // expected (the first launch's phases carry tags 1, 2, ...)
-        cudaError_t e = cudaMemsetAsync(c->arena + c->lay.ctl, 0, (size_t)kCtlWords * 8, c->stream);
-        if (e == cudaSuccess) e = cudaMemsetAsync(c->arena + c->lay.x, 0, c->lay.part - c->lay.x, c->stream);
+        // Control words, the split-K buffers and the tagged words start at zero: tag 0 is
+        // never expected (the first launch's phases carry tags 1, 2, ...).
+        cudaError_t e = cudaMemsetAsync(c->arena + c->lay.delta, 0, c->lay.ctl + (size_t)kCtlWords * 8 - c->lay.delta,
+                                        c->stream);
         if (e != cudaSuccess) rc = fail(c, KD_ECUDA, "cudaMemsetAsync: %s", cudaGetErrorString(e));
     }
     if (rc != KD_OK) {
@@ -317,15 +360,19 @@ int kd_load_weights(kd_ctx* c, const kd_weights* w) {
     };
     KD_CUDA(c, per_layer(y.l_attn_norm, w->attn_norm, D * 2));
     KD_CUDA(c, per_layer(y.l_ffn_norm, w->ffn_norm, D * 2));
-    KD_CUDA(c, per_layer(y.l_wo, w->wo, D * d.qd * 2));
-    KD_CUDA(c, per_layer(y.l_wd, w->wd, D * d.F * 2));
     repack_qkv<<<dim3(d.qkv_rows, d.L), 128, 0, s>>>(l0, y.layer_stride, y.l_wqkv, (const uint16_t*)w->wq,
                                                       (const uint16_t*)w->wk, (const uint16_t*)w->wv, d);
     KD_CUDA(c, cudaGetLastError());
     repack_gu<<<dim3(2 * d.F, d.L), 128, 0, s>>>(l0, y.layer_stride, y.l_wgu, (const uint16_t*)w->wg,
                                                   (const uint16_t*)w->wu, d);
     KD_CUDA(c, cudaGetLastError());
-    c->launches += 2;
+    transpose_bf16<<<dim3((d.qd + 31) / 32, (d.d + 31) / 32, d.L), dim3(32, 8), 0, s>>>(
+        l0, y.layer_stride, y.l_wot, (const uint16_t*)w->wo, d.d, d.qd);
+    KD_CUDA(c, cudaGetLastError());
+    transpose_bf16<<<dim3((d.F + 31) / 32, (d.d + 31) / 32, d.L), dim3(32, 8), 0, s>>>(
+        l0, y.layer_stride, y.l_wdt, (const uint16_t*)w->wd, d.d, d.F);
+    KD_CUDA(c, cudaGetLastError());
+    c->launches += 4;
     // RoPE table: (cos, sin) of position p times frequency theta^(-2i/hd), formed in double
     // and rounded to float, for every position the cache can hold; the kernel reads one row
     // per step.
@@ -368,10 +415,12 @@ void* kd_kv_ptr(kd_ctx* c, int32_t layer, int32_t which) {
 static int reset_common(kd_ctx* c, int32_t n_tokens, int32_t kv_len) {
     if (n_tokens < 1 || kv_len < 0 || kv_len >= c->dm.S || n_tokens > c->dm.S)
         return fail(c, KD_EINVAL, "kd_reset: need n_tokens >= 1 and 0 <= kv_len < max_seq");
-    // Control words are left consistent by every completed launch (the kernel re-bases
-    // its barrier count and clears its own argmax slots), so they are cleared only after a
-    // failed run: the decode path then involves no memset.
-    if (c->failed) KD_CUDA(c, cudaMemsetAsync(c->arena + c->lay.ctl, 0, (size_t)kCtlWords * 8, c->stream));
+    // Every completed launch leaves the control words and the split-K buffers consistent
+    // (the kernel re-bases its sync count, clears its argmax slots and zeroes the buffers), so
+    // they are cleared only after a failed run: the decode path then involves no memset.
+    if (c->failed)
+        KD_CUDA(c, cudaMemsetAsync(c->arena + c->lay.delta, 0, c->lay.ctl + (size_t)kCtlWords * 8 - c->lay.delta,
+                                   c->stream));
     c->pos = kv_len;
     c->n_pending = n_tokens;
     c->failed = false;
@@ -387,6 +436,7 @@ int kd_reset(kd_ctx* c, const int32_t* d_tokens, int32_t n_tokens, int32_t kv_le
     return KD_OK;
 }
 
+
 int kd_decode(kd_ctx* c, int32_t n_gen, int32_t* d_tokens_out, float* d_logits_out) {
     if (!c) return KD_EINVAL;
     if (!c->has_weights || c->n_pending < 1) return fail(c, KD_ESTATE, "kd_decode: no weights or nothing pending");
@@ -396,10 +446,12 @@ int kd_decode(kd_ctx* c, int32_t n_gen, int32_t* d_tokens_out, float* d_logits_o
     if (steps == 0) return KD_OK;
     if ((long long)c->pos + steps > c->dm.S)
         return fail(c, KD_ECAPACITY, "kd_decode: position %d + %d steps exceeds max_seq %d", c->pos, steps, c->dm.S);
+    kd_ctx_view v;
+    kd_internal_view(c, &v);
     Params p{};
+    fill_launch_shape(v, p);
     p.arena = c->arena;
     p.lay = c->lay;
-    p.dm = c->dm;
     p.steps = steps;
     p.n_pending = c->n_pending;
     p.pos0 = c->pos;
@@ -407,20 +459,6 @@ int kd_decode(kd_ctx* c, int32_t n_gen, int32_t* d_tokens_out, float* d_logits_o
     p.dump = d_logits_out != nullptr;
     p.tokens_out = d_tokens_out;
     p.logits_out = d_logits_out;
-    p.nb = c->nb;
-    p.ns = c->ns;
-    p.attn_pieces = c->pieces;
-    p.pos_per_stage = c->pos_per_stage;
-    p.rows_qkv = rows_per_stage(c->dm.d, true);
-    p.rows_o = rows_per_stage(c->dm.qd, false);
-    p.rows_gu = rows_per_stage(c->dm.d, true);
-    p.rows_d = rows_per_stage(c->dm.F, false);
-    p.rows_lm = rows_per_stage(c->dm.d, false);
-    p.xs_floats = c->xs_floats;
-    p.xown_floats = c->xown_floats;
-    p.timeout_ns = c->timeout_ns;
-    p.prefetch = c->prefetch;
-    p.inflight = c->inflight;
     p.tag0 = c->tag;
     p.trace = c->trace;
     p.trace_every = c->trace_every;
@@ -429,7 +467,7 @@ int kd_decode(kd_ctx* c, int32_t n_gen, int32_t* d_tokens_out, float* d_logits_o
     launch_decode(p, c->stream, c->smem, &e);
     if (e != 0) return fail(c, KD_ECUDA, "cooperative launch failed: %s", cudaGetErrorString((cudaError_t)e));
     c->launches += 1;
-    c->tag += (uint32_t)launch_phases(c->dm, steps, c->n_pending, d_logits_out != nullptr);
+    c->tag += (uint32_t)launch_tags(c->dm.L, steps);
     c->pos += steps;
     c->n_pending = 1;
     return KD_OK;
@@ -504,6 +542,7 @@ int kd_get_info(const kd_ctx* c, kd_info* info) {
     info->weight_bytes = (int64_t)c->lay.weights_end;
     info->kv_bytes = (int64_t)c->lay.kv_bytes;
     info->launches = c->launches;
+    info->ctl_offset = (int64_t)c->lay.ctl;
     return KD_OK;
 }
 

@@ -1,34 +1,36 @@
 // kd_layout.h -- arena layout, launch constants and kernel parameters shared by the host
-// side of libkd (kd_api.cu) and the monokernel (kd_kernel.cu). Internal to libkd.
+// side of libkd (kd_api.cu, kd_noalloc.cu) and the monokernel (kd_kernel.cu). Internal to libkd.
 #pragma once
 
 #include <stddef.h>
 #include <stdint.h>
 
+#ifdef __CUDACC__
+#define KD_HD __host__ __device__
+#else
+#define KD_HD
+#endif
+
 namespace kd {
 
-// Pipeline: one producer warp streams weight / KV tiles into a ring of shared-memory
-// stages with 1-D bulk copies; consumer warps each take whole stages round-robin.
+// One CTA per SM: one producer warp streams weight / KV tiles into a ring of shared-memory
+// stages with 1-D bulk copies; 16 consumer warps share every stage.
 constexpr int kStageBytes = 32768;
-constexpr int kGroupWarps = 8;                      // warps that share one pipeline stage
-constexpr int kGroups = 1;                          // groups take alternate stages (slot parity)
-constexpr int kConsumerWarps = kGroupWarps * kGroups;  // + 1 producer warp
+constexpr int kConsumerWarps = 16;
 constexpr int kConsumerThreads = 32 * kConsumerWarps;
 constexpr int kThreads = kConsumerThreads + 32;
-constexpr int kMaxRows = 8;       // rows of one GEMV stage (one per warp of a group)
-constexpr int kMaxChunks = 8;     // 16-byte weight chunks per lane per row slice (x kept in registers)
-constexpr int kMaxGroup = 8;      // q heads per kv head
-constexpr int kMaxKvHeads = 16;
 constexpr int kMaxStages = 8;
+constexpr int kMaxGroup = 8;        // q heads per kv head
+constexpr int kMaxKvHeads = 16;
+constexpr int kMaxModel = 8192;     // d_model
 constexpr int kSmemLimit = 232448;  // opt-in dynamic shared memory per CTA on B200
 
 // Control words (uint64), each on its own 128-byte line.
-constexpr int kCtlBar = 0;                 // grid-barrier arrivals, monotonic
-constexpr int kCtlStatus = 16;             // 0 = ok, else an error code (device side)
-constexpr int kCtlWhere = 17;              // where a wait gave up (debug)
-constexpr int kCtlArgmax = 32;             // 3 argmax slots at kCtlArgmax + 16*i
-constexpr int kCtlHead = 96;               // split-K arrival counters at kCtlHead + 16*g
-constexpr int kCtlWords = kCtlHead + 16 * kMaxKvHeads;
+constexpr int kCtlSync = 0;     // arrivals at the cross-CTA sums and the argmax, monotonic
+constexpr int kCtlStatus = 16;  // 0 = ok, else an error code (device side)
+constexpr int kCtlWhere = 17;   // where a wait gave up (diagnosis)
+constexpr int kCtlArgmax = 32;  // 3 rotating argmax slots at kCtlArgmax + 16*i
+constexpr int kCtlWords = 80;
 
 constexpr int kStatusTimeout = 1;  // a device-side wait exceeded its limit
 constexpr int kStatusToken = 2;    // a token id outside [0, vocab) reached the kernel
@@ -44,57 +46,74 @@ struct Dims {
 struct Layout {
     size_t embed, lm_head, final_norm;
     size_t layer0, layer_stride;
-    size_t l_attn_norm, l_ffn_norm, l_wqkv, l_wo, l_wgu, l_wd;  // within a layer block
-    size_t rope;                                                  // [S][hd/2] float2 (cos, sin)
-    size_t kcache, vcache;                                        // [L][Hkv][S][hd] bf16
-    // Activations exchanged between CTAs, each element a 64-bit word (fp32 value in the low
-    // half, the producing phase's tag in the high half): x [2][d] (outputs of O and of D),
-    // qkv [qkv_rows], o [qd], gu [F] (the FFN hidden vector). Attention partials are fp32.
-    size_t x, qkv, o, gu, part;
+    // within a layer block: the two norm gains, then the matrices in streaming order:
+    //   wqkv [Hkv][(r + 2) * hd][d]  per kv head: its r q heads, its k head, its v head; q and k
+    //                                rows in RoPE-pair order (row 2i = dim i, 2i + 1 = dim i + hd/2)
+    //   wot  [Hq * hd][d]            the output projection transposed (row = attention dim)
+    //   wgu  [2F][d]                 gate and up rows interleaved (2j = gate j, 2j + 1 = up j)
+    //   wdt  [F][d]                  the down projection transposed (row = hidden unit)
+    size_t l_attn_norm, l_ffn_norm, l_wqkv, l_wot, l_wgu, l_wdt;
+    size_t rope;            // [S][hd/2] float2 (cos, sin)
+    size_t kcache, vcache;  // [L][Hkv][S][hd] bf16
+    // Scratch written during a launch:
+    //   delta [3][d] fp32  -- cross-CTA sums of the split-K output and down projections
+    //   qkv [Hkv][(r + 2) * hd] tagged words -- RoPE'd q, RoPE'd bf16 k, bf16 v of the step
+    //   rec [grid][r][hd + 2] tagged words   -- attention piece records (max, sum, acc[hd])
+    size_t delta, qkv, rec;
     size_t ctl, tokens_in, tokens_out;
     size_t weights_end, kv_bytes, total;
 };
 
-// Rows per pipeline stage of one GEMV phase with reduction length K (bf16 elements): the
-// largest power of two <= 8 whose rows fit a stage. The kernel cuts each row into slices
-// (16 / R of them when R >= 2, else 8) shared by the 8 consumer warps.
-inline int rows_per_stage(int K, bool paired) {
-    int r = kStageBytes / (2 * K);
-    if (r > kMaxRows) r = kMaxRows;
-    int p2 = 1;
-    while (p2 * 2 <= r) p2 *= 2;
-    (void)paired;
-    return p2;
+// Shapes of the two GEMV kinds for a model of width d (both stream rows of d bf16 elements):
+//  row GEMV (Q/K/V, gate/up, LM head): a row is cut into gs slices of at most 1024 elements
+//    (4 chunks of 8 per lane), a stage holds gr rows, and the 16 consumer warps share the
+//    gr * gs (row, slice) units of a stage, gm = gr * gs / 16 each;
+//  split-K GEMV (output and down projections): a stage holds kr rows; thread t owns the
+//    8 outputs of chunk t % (d / 8) and the rows t / (d / 8) + k * ug of each stage.
+struct Shape {
+    int gs, gr, gm;  // row GEMV
+    int kr, ug, kc;  // split-K GEMV: rows per stage, unit groups, output chunks per thread
+};
+inline bool make_shape(int d, Shape* s) {
+    if (d < 256 || d % 256 || d > kMaxModel) return false;
+    int gs = 1;
+    while (d / gs > 1024) gs *= 2;
+    if ((d / gs) % 256) return false;
+    const int maxr = kStageBytes / (2 * d);
+    const int unit = kConsumerWarps / gs;  // rows must come in multiples of this
+    int gr = (maxr / unit) * unit;
+    if (gr > 64) gr = 64;
+    if (gr < unit) return false;
+    s->gs = gs;
+    s->gr = gr;
+    s->gm = gr * gs / kConsumerWarps;
+    if (s->gm != 1 && s->gm != 2 && s->gm != 4) return false;
+    const int oc = d / 8;
+    s->kr = maxr > 64 ? 64 : maxr;
+    s->ug = oc >= kConsumerThreads ? 1 : kConsumerThreads / oc;
+    s->kc = (oc + kConsumerThreads - 1) / kConsumerThreads;
+    if (s->kc > 2) return false;
+    return true;
 }
 
-// Chunks of 8 elements per lane that a GEMV slice of reduction length K needs when a stage
-// holds R = rows_per_stage(K) rows cut into 16 / R slices (R >= 2) or 8 slices (R == 1).
-inline int gemv_slice_chunks(int K) {
-    const int R = rows_per_stage(K, false);
-    const int slices = R >= 2 ? 16 / R : 8;
-    return (K / slices + 255) / 256;
+// Cross-CTA sums ("syncs") per decode step: the output projection and the down projection of
+// every layer, then the argmax of the steps that run the LM head (all steps when logits are
+// dumped). Sync k adds into delta buffer k % 3.
+KD_HD inline long long syncs_before_step(int L, int s, int n_pending, bool dump) {
+    const long long heads = dump ? s : (s - (n_pending - 1) > 0 ? s - (n_pending - 1) : 0);
+    return 2LL * L * s + heads;
 }
-inline int gemv_max_chunks(const Dims& dm) {
-    int m = gemv_slice_chunks(dm.d);
-    if (gemv_slice_chunks(dm.qd) > m) m = gemv_slice_chunks(dm.qd);
-    if (gemv_slice_chunks(dm.F) > m) m = gemv_slice_chunks(dm.F);
-    return m;
-}
-
-// Phases one launch runs: per step 5 per layer (QKV, ATT, O, GU, D), plus the LM head at
-// the steps that pick a token (or at every step when logits are dumped). Tags of
-// successive launches follow each other, so a buffer element never carries a stale tag
-// that a reader of a later launch expects.
-inline long long launch_phases(const Dims& dm, int steps, int n_pending, bool dump) {
-    const long long heads = dump ? steps : (steps - (n_pending - 1) > 0 ? steps - (n_pending - 1) : 0);
-    return (long long)steps * 5 * dm.L + heads;
-}
+// Tagged phases (Q/K/V outputs and attention records) a launch of `steps` steps writes: two per
+// layer and step. Tags of successive launches follow each other, so a word never carries a
+// stale tag that a reader of a later launch expects.
+KD_HD inline long long launch_tags(int L, int steps) { return 2LL * L * steps; }
 
 struct Params {
     // weights (arena)
     const uint8_t* arena;
     Layout lay;
     Dims dm;
+    Shape sh;
     // per-launch
     int steps;      // decode steps in this launch
     int n_pending;  // tokens fed before the first generated one
@@ -104,27 +123,23 @@ struct Params {
     int32_t* tokens_out;
     float* logits_out;
     // launch shape
-    int nb;           // CTAs
-    int ns;           // pipeline stages
-    int attn_pieces;  // CTAs per kv head in attention
-    int pos_per_stage;
-    int rows_qkv, rows_o, rows_gu, rows_d, rows_lm;  // rows per stage of each GEMV phase
-    int xs_floats;                                    // activation buffer (floats)
-    int xown_floats;                                  // this CTA's residual rows (floats)
+    int nb;         // CTAs
+    int ns;         // pipeline stages
+    int pieces;     // CTAs per kv head (attention pieces, and the Q/K/V and output-projection shares)
+    int blk;        // positions per attention softmax block
+    int work_floats, hin_floats;  // shared-memory scratch sizes
     long long timeout_ns;
-    int prefetch;  // stages the producer pulls into L2 ahead of the shared-memory ring
-    int inflight;  // at most this many issued stages not yet landed (bounds memory queueing)
-    uint32_t tag0;  // phase i of this launch tags its outputs tag0 + 1 + i (see kd_kernel.cu)
+    uint32_t tag0;  // tagged phase i of this launch tags its words tag0 + 1 + i
     // optional trace: CTAs with blockIdx.x % trace_every == 0 record per-phase timestamps
     unsigned long long* trace;
-    int trace_every, trace_rows;  // rows per traced CTA (4 words each)
+    int trace_every, trace_rows;
 };
 
-// Trace row layout (SM clock cycles): consumer rows [begin, loaded, arrive, done, s4..s7] per
-// phase, in phase order, where s4..s7 are attention sub-steps (q loaded, cache pieces done,
-// partial record written, combine done; 0 elsewhere); the last row of a traced CTA holds the
-// producer's [cycles blocked on a free slot, cycles blocked on a KV epoch, stages issued,
-// total cycles].
+// Trace row layout (SM clock cycles), one row per phase of a traced CTA, in phase order:
+// [phase id (step << 16 | layer << 4 | phase), begin, inputs ready, compute done, end,
+//  cycles waiting for weight / KV stages, 0, 0]. The last row of a traced CTA holds the
+// producer warp's [cycles waiting for a free stage, cycles waiting for KV rows written this
+// launch, stages issued, total cycles].
 constexpr int kTraceWords = 8;
 
 void launch_decode(const Params& p, void* stream, int smem_bytes, int* err);
@@ -133,11 +148,11 @@ void launch_decode(const Params& p, void* stream, int smem_bytes, int* err);
 struct kd_ctx_view {
     const Dims* dm;
     const Layout* lay;
+    const Shape* sh;
     uint8_t* arena;
     void* stream;
-    int device, nb, smem, ns, pieces, pos_per_stage, xs_floats, xown_floats;
+    int device, nb, smem, ns, pieces, blk, work_floats, hin_floats;
     long long timeout_ns;
-    int prefetch, inflight;
     bool has_weights;
 };
 int monokernel_smem_bytes(const Params& p);

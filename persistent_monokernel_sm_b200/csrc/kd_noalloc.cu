@@ -19,6 +19,9 @@
 using namespace kd;
 
 int kd_internal_view(kd_ctx* ctx, kd_ctx_view* v);
+namespace kd {
+void fill_launch_shape(const kd_ctx_view& v, Params& p);
+}
 int kd_internal_fail(kd_ctx* ctx, int code, const char* msg);
 void kd_internal_count_launch(kd_ctx* ctx);
 
@@ -70,9 +73,9 @@ extern "C" int kd_decode_noalloc(kd_ctx* ctx, const int32_t* d_tokens, int32_t n
         off = up256(off + bytes);
         return at;
     };
-    const size_t o_x = take((size_t)2 * dm.d * 8), o_q = take((size_t)dm.qkv_rows * 8), o_o = take((size_t)dm.qd * 8);
-    const size_t o_hdn = take((size_t)dm.F * 8);
-    const size_t o_part = take((size_t)v.nb * dm.r * (dm.hd + 2) * 4);
+    const size_t o_delta = take((size_t)3 * dm.d * 4);
+    const size_t o_qkv = take((size_t)dm.qkv_rows * 8);
+    const size_t o_rec = take((size_t)v.nb * dm.r * (dm.hd + 2) * 8);
     const size_t o_ctl = take((size_t)kCtlWords * 8);
     const size_t o_tok = take((size_t)n_tokens * 4);
     if (off > kNoallocScratchBytes) {
@@ -92,11 +95,10 @@ extern "C" int kd_decode_noalloc(kd_ctx* ctx, const int32_t* d_tokens, int32_t n
         return kd_internal_fail(ctx, KD_ECUDA, cudaGetErrorString(e));
     uint8_t* s = static_cast<uint8_t*>(base);
 
-    // Control words and the tagged activation words must start at zero (the array keeps the
-    // previous call's contents, possibly another handle's, so tags restart at 1 each call);
-    // the pending tokens are copied in. None of this allocates.
-    if ((e = cudaMemsetAsync(s + o_ctl, 0, (size_t)kCtlWords * 8, (cudaStream_t)v.stream)) != cudaSuccess ||
-        (e = cudaMemsetAsync(s + o_x, 0, o_part - o_x, (cudaStream_t)v.stream)) != cudaSuccess ||
+    // The split-K buffers, tagged words and control words must start at zero (the array keeps
+    // the previous call's contents, possibly another handle's, so tags restart at 1 each
+    // call); the pending tokens are copied in. None of this allocates.
+    if ((e = cudaMemsetAsync(s + o_delta, 0, o_tok - o_delta, (cudaStream_t)v.stream)) != cudaSuccess ||
         (e = cudaMemcpyAsync(s + o_tok, d_tokens, (size_t)n_tokens * 4, cudaMemcpyDeviceToDevice, (cudaStream_t)v.stream)) !=
             cudaSuccess)
         return kd_internal_fail(ctx, KD_ECUDA, cudaGetErrorString(e));
@@ -106,11 +108,11 @@ extern "C" int kd_decode_noalloc(kd_ctx* ctx, const int32_t* d_tokens, int32_t n
     // relative to the arena so that they land in the array (64-bit wrap-around addition).
     auto rel = [&](size_t o) { return (size_t)((uintptr_t)(s + o) - (uintptr_t)v.arena); };
     Params p{};
+    fill_launch_shape(v, p);
     p.arena = v.arena;
     p.lay = *v.lay;
-    p.lay.x = rel(o_x), p.lay.qkv = rel(o_q), p.lay.o = rel(o_o), p.lay.gu = rel(o_hdn);
-    p.lay.part = rel(o_part), p.lay.ctl = rel(o_ctl), p.lay.tokens_in = rel(o_tok);
-    p.dm = dm;
+    p.lay.delta = rel(o_delta), p.lay.qkv = rel(o_qkv), p.lay.rec = rel(o_rec);
+    p.lay.ctl = rel(o_ctl), p.lay.tokens_in = rel(o_tok);
     p.steps = steps;
     p.n_pending = n_tokens;
     p.pos0 = kv_len;
@@ -118,20 +120,6 @@ extern "C" int kd_decode_noalloc(kd_ctx* ctx, const int32_t* d_tokens, int32_t n
     p.dump = d_logits_out != nullptr;
     p.tokens_out = d_tokens_out;
     p.logits_out = d_logits_out;
-    p.nb = v.nb;
-    p.ns = v.ns;
-    p.attn_pieces = v.pieces;
-    p.pos_per_stage = v.pos_per_stage;
-    p.rows_qkv = rows_per_stage(dm.d, true);
-    p.rows_o = rows_per_stage(dm.qd, false);
-    p.rows_gu = rows_per_stage(dm.d, true);
-    p.rows_d = rows_per_stage(dm.F, false);
-    p.rows_lm = rows_per_stage(dm.d, false);
-    p.xs_floats = v.xs_floats;
-    p.xown_floats = v.xown_floats;
-    p.timeout_ns = v.timeout_ns;
-    p.prefetch = v.prefetch;
-    p.inflight = v.inflight;
     p.tag0 = 0;
     int err = 0;
     launch_decode(p, v.stream, v.smem, &err);

@@ -23,6 +23,12 @@ import numpy as np
 ATOL = 2e-2
 REL_L2 = 1e-3
 MARGIN = 5e-2
+# Two launches of the same request differ only in the order of the fp32 atomic additions
+# that sum the split-K output and down projections (a few ulps per layer): their logits
+# agree far inside the parity tolerance, and their tokens agree except where the top two
+# logits are closer than that noise.
+RUN_REL_L2 = 1e-5
+RUN_MARGIN = 1e-3
 
 
 def oracle_threads() -> int:
@@ -87,3 +93,23 @@ def compare_free_run(gpu_tokens, gpu_logits, ref_tokens, ref_logits, what: str =
             assert lg[int(gpu_tokens[i])] >= lg.max() - MARGIN
             return i + 1
     return n
+
+
+def compare_gpu_runs(toks_a, toks_b, logits_a, what: str = "", logits_b=None):
+    """Two GPU launches of the same request (same weights, inputs and positions). Their
+    tokens must agree up to the first step whose top-1/top-2 margin (in run a) is below
+    RUN_MARGIN, where the order of the atomic additions may decide a near-tie; while the
+    histories agree, the logits (when both are given) must agree within RUN_REL_L2.
+    Returns the number of steps that agree."""
+    toks_a = np.asarray(toks_a)
+    toks_b = np.asarray(toks_b)
+    assert toks_a.shape == toks_b.shape
+    for i in range(len(toks_a)):
+        if logits_b is not None:
+            rel = float(rel_l2(logits_b[i:i + 1], logits_a[i:i + 1])[0])
+            assert rel <= RUN_REL_L2, "%s: step %d runs differ by rel-L2 %.3g" % (what, i, rel)
+        if int(toks_a[i]) != int(toks_b[i]):
+            m = margin(logits_a[i])
+            assert m < RUN_MARGIN, "%s: runs diverge at step %d with margin %.3g" % (what, i, m)
+            return i
+    return len(toks_a)
