@@ -183,7 +183,8 @@ int kd_decode_noalloc(kd_ctx *ctx, const int32_t *d_tokens, int32_t n_tokens, in
  * output projection, gate/up, down, LM head) and in phase order, a row of eight words:
  * the phase id (step << 16 | layer << 4 | phase 0..5), then SM-clock stamps of phase begin,
  * inputs ready (the cross-CTA sync passed or the tagged inputs polled), compute done and
- * phase end, then the cycles spent waiting for weight / KV stages, then two zero words.
+ * phase end, then the cycles spent waiting for weight / KV stages, then the stamps of the
+ * phase's first and last weight / KV stage becoming ready (0 in a phase without stages).
  * Traced CTA i owns rows [i * R, (i + 1) * R) of the buffer, where
  * R = n_words / (8 * ceil(grid / every)); its last row holds the producer warp's cycles
  * blocked on a free pipeline stage, cycles blocked on KV rows written during the launch,

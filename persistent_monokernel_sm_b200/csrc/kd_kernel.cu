@@ -116,6 +116,9 @@ __device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, 
                  "f"(d)
                  : "memory");
 }
+__device__ __forceinline__ void red_max_u64(unsigned long long* p, unsigned long long v) {
+    asm volatile("red.relaxed.gpu.global.max.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
 __device__ __forceinline__ float4 ld_relaxed_v4(const float* p) {
     float4 v;
     asm volatile("ld.relaxed.gpu.global.v4.f32 {%0, %1, %2, %3}, [%4];"
@@ -124,6 +127,12 @@ __device__ __forceinline__ float4 ld_relaxed_v4(const float* p) {
                  : "memory");
     return v;
 }
+
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 // Tagged activation words: value (fp32 bits) in the low half, the producing phase's tag in
 // the high half. A 64-bit store is single-copy atomic, so a reader that sees the tag sees
@@ -202,8 +211,15 @@ struct Tracer {
     __device__ __forceinline__ void begin(int id) {
         if (row0 && row < rows - 1) {
             row0[(size_t)row * kTraceWords] = (unsigned long long)id;
+            row0[(size_t)row * kTraceWords + 6] = 0ull;
+            row0[(size_t)row * kTraceWords + 7] = 0ull;
             mark(1);
         }
+    }
+    // stage j of nst of the phase has landed: the first and the last one are stamped
+    __device__ __forceinline__ void stage_ready(int j, int nst) {
+        if (j == 0) mark(6);
+        if (j == nst - 1) mark(7);
     }
     __device__ __forceinline__ void end() {
         if (row0 && row < rows - 1) {
@@ -293,6 +309,7 @@ __device__ __forceinline__ uint32_t qkv_tag(const Params& P, int t, int l) {
 struct Smem {
     uint8_t* ring;            // ns * kStageBytes
     float* x;                 // the residual stream (d), identical in every CTA
+    __nv_bfloat16* gain;      // the norm gain of the next row GEMV (d), prefetched
     float* hin;               // split-K inputs: this CTA's hidden values or attention output dims
     float* work;              // GEMV row partials / attention scores and reductions / split-K sums
     float* qs;                // attention: q of the kv head's q heads (r * hd), prescaled
@@ -310,7 +327,7 @@ struct Smem {
 // Byte offsets of the shared-memory regions; the ring starts at 0 (1024-aligned), the others
 // on 128-byte boundaries. Used by the kernel and for the launch size.
 struct SmemLayout {
-    size_t ring, x, hin, work, qs, kvc, rope, red, stats, u64, flag, full, empty, geo, total;
+    size_t ring, x, gain, hin, work, qs, kvc, rope, red, stats, u64, flag, full, empty, geo, total;
 };
 __host__ __device__ inline SmemLayout smem_layout(int ns, int d, int hd, int r, int hin_floats, int work_floats) {
     SmemLayout L{};
@@ -322,6 +339,7 @@ __host__ __device__ inline SmemLayout smem_layout(int ns, int d, int hd, int r, 
     };
     L.ring = take((size_t)ns * kStageBytes);
     L.x = take((size_t)d * 4);
+    L.gain = take((size_t)d * 2);
     L.hin = take((size_t)hin_floats * 4);
     L.work = take((size_t)work_floats * 4);
     L.qs = take((size_t)r * hd * 4);
@@ -343,6 +361,7 @@ __device__ __forceinline__ Smem carve(const Params& P, uint8_t* base) {
     Smem s;
     s.ring = base + L.ring;
     s.x = reinterpret_cast<float*>(base + L.x);
+    s.gain = reinterpret_cast<__nv_bfloat16*>(base + L.gain);
     s.hin = reinterpret_cast<float*>(base + L.hin);
     s.work = reinterpret_cast<float*>(base + L.work);
     s.qs = reinterpret_cast<float*>(base + L.qs);
@@ -377,22 +396,33 @@ struct Ring {
     }
 };
 
-// Wait (whole warp) for the stage in `rg` to land. `waited` accumulates the cycles (trace).
+// Wait (whole warp) for the stage in `rg` to land. Only lane 0 polls the mbarrier (sixteen
+// warps times 32 lanes polling one shared-memory word would serialise on it); the shuffle
+// hands its answer to the warp and the warp barrier orders the other lanes' reads of the
+// stage after lane 0's observation of the completed phase. `waited` accumulates the cycles
+// spent (trace).
 __device__ __forceinline__ bool wait_full(const Smem& sm, const Ring& rg, const Params& P, const unsigned long long* ctl,
                                           unsigned long long& waited) {
     const uint32_t a = smem_u32(&sm.full[rg.slot]);
-    if (__all_sync(0xffffffffu, mbar_try_wait(a, rg.phase))) return true;
-    const long long c0 = clock64();
-    Deadline dl;
-    for (;;) {
-        if (__all_sync(0xffffffffu, mbar_wait_hint(a, rg.phase))) {
-            waited += (unsigned long long)(clock64() - c0);
-            return true;
+    int done = 0;
+    if ((threadIdx.x & 31) == 0) {
+        done = mbar_try_wait(a, rg.phase);
+        if (!done) {
+            const long long c0 = clock64();
+            Deadline dl;
+            for (;;) {
+                if (mbar_wait_hint(a, rg.phase)) {
+                    done = 1;
+                    waited += (unsigned long long)(clock64() - c0);
+                    break;
+                }
+                if (!dl.alive(ctl, P.timeout_ns, where_code(kWhereFull, rg.slot))) break;
+            }
         }
-        int bad = 0;
-        if ((threadIdx.x & 31) == 0) bad = !dl.alive(ctl, P.timeout_ns, where_code(kWhereFull, rg.slot));
-        if (__shfl_sync(0xffffffffu, bad, 0)) return false;
     }
+    done = __shfl_sync(0xffffffffu, done, 0);
+    __syncwarp();
+    return done != 0;
 }
 // The warp is done with the stage: one arrival per warp on the slot's empty barrier.
 __device__ __forceinline__ void release(const Smem& sm, const Ring& rg) {
@@ -426,22 +456,18 @@ __device__ __forceinline__ void sync_arrive(unsigned long long* ctl) {
 // Wait until every CTA has arrived at this launch's sync number k (thread 0 polls with
 // acquire loads, the CTA barrier then orders every consumer thread after it). Returns
 // false in every consumer thread when the wait gave up or another wait failed.
+__device__ __noinline__ int sync_spin(const unsigned long long* ctl, uint64_t target, long long timeout_ns, long long k) {
+    Deadline dl;
+    for (uint32_t it = 0;; ++it) {
+        if (ld_acquire_u64(ctl + kCtlSync) >= target) return 1;
+        if ((it & 31) == 31 && !dl.alive(ctl, timeout_ns, where_code(kWhereSync, (int)(k & 0xff)))) return 0;
+    }
+}
 __device__ __forceinline__ bool sync_wait(const Smem& sm, const Params& P, const unsigned long long* ctl, long long k,
                                           bool ok) {
     if (threadIdx.x == 0) {
-        int good = ok ? 1 : 0;
         const uint64_t target = sm.u64[0] + (uint64_t)(k + 1) * (uint64_t)P.nb;
-        if (good && ld_acquire_u64(ctl + kCtlSync) < target) {
-            Deadline dl;
-            for (uint32_t it = 0;; ++it) {
-                if (ld_acquire_u64(ctl + kCtlSync) >= target) break;
-                if ((it & 31) == 31 && !dl.alive(ctl, P.timeout_ns, where_code(kWhereSync, (int)(k & 0xff)))) {
-                    good = 0;
-                    break;
-                }
-            }
-        }
-        sm.flag[0] = good;
+        sm.flag[0] = ok ? sync_spin(ctl, target, P.timeout_ns, k) : 0;
     }
     consumer_sync();
     return sm.flag[0] != 0;
@@ -458,41 +484,43 @@ __device__ __forceinline__ void zero_previous(const Params& P, long long k) {
     const int z0 = (int)((long long)d * blockIdx.x / P.nb), z1 = (int)((long long)d * (blockIdx.x + 1) / P.nb);
     for (int i = z0 + (int)threadIdx.x; i < z1; i += kConsumerThreads) old[i] = 0.f;
 }
-// After sync k has completed: fold delta buffer k % 3 (the sum of every CTA's split-K
-// partials) into the residual stream, and recycle the previous buffer.
-__device__ __forceinline__ void fold_delta(const Smem& sm, const Params& P, long long k) {
-    const int d = P.dm.d;
-    const float* src = reinterpret_cast<const float*>(P.arena + P.lay.delta) + (size_t)(k % 3) * d;
-    for (int i = threadIdx.x * 4; i < d; i += kConsumerThreads * 4) {
-        const float4 v = ld_relaxed_v4(src + i);
-        float4* xp = reinterpret_cast<float4*>(sm.x + i);
-        float4 x = *xp;
-        x.x += v.x, x.y += v.y, x.z += v.z, x.w += v.w;
-        *xp = x;
-    }
-    zero_previous(P, k);
-    consumer_sync();
+// Start copying the norm gain of the coming row GEMV into shared memory (asynchronously:
+// it lands while the phase waits for its inputs). fold_norm waits for it.
+__device__ __forceinline__ void prefetch_gain(const Smem& sm, const __nv_bfloat16* gain, int d) {
+    for (int i = threadIdx.x; i < d / 8; i += kConsumerThreads) cp_async16(sm.gain + i * 8, gain + i * 8);
+    cp_async_commit();
 }
 
-// ------------------------------------------------------------------ RMSNorm scale
-
-// 1 / sqrt(mean(x^2) + eps) of the residual stream in shared memory. Every CTA sums the
-// same values in the same order, so all of them get the same scale.
-__device__ __forceinline__ float rms_scale(const Smem& sm, int d, float eps) {
+// The residual stream's update and its RMSNorm scale. With k >= 0 (sync k has completed),
+// delta buffer k % 3 -- the sum of every CTA's split-K partials -- is folded into the
+// residual first, and this CTA's slice of the previous buffer is recycled. Returns
+// 1 / sqrt(mean(x^2) + eps) of the result: every CTA sums the same values in the same
+// order, so all of them get the same scale. Also completes the gain prefetch.
+__device__ __forceinline__ float fold_norm(const Smem& sm, const Params& P, long long k) {
+    const int d = P.dm.d;
+    const float* src = reinterpret_cast<const float*>(P.arena + P.lay.delta) + (size_t)(k >= 0 ? k % 3 : 0) * d;
     float ss = 0.f;
     for (int i = threadIdx.x * 4; i < d; i += kConsumerThreads * 4) {
-        const float4 v = *reinterpret_cast<const float4*>(sm.x + i);
-        ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+        float4* xp = reinterpret_cast<float4*>(sm.x + i);
+        float4 x = *xp;
+        if (k >= 0) {
+            const float4 v = ld_relaxed_v4(src + i);
+            x.x += v.x, x.y += v.y, x.z += v.z, x.w += v.w;
+            *xp = x;
+        }
+        ss += x.x * x.x + x.y * x.y + x.z * x.z + x.w * x.w;
     }
+    if (k >= 0) zero_previous(P, k);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
     if ((threadIdx.x & 31) == 0) sm.red[threadIdx.x >> 5] = ss;
+    cp_async_wait_all();
     consumer_sync();
-    float tot = 0.f;
-#pragma unroll
-    for (int w = 0; w < kConsumerWarps; ++w) tot += sm.red[w];
-    consumer_sync();  // red is reused
-    return 1.0f / sqrtf(tot / (float)d + eps);
+    const float4* r4 = reinterpret_cast<const float4*>(sm.red);
+    const float4 a = r4[0], b = r4[1], c = r4[2], e = r4[3];  // the 16 warp sums, read at once
+    const float tot = ((a.x + a.y) + (a.z + a.w)) + ((b.x + b.y) + (b.z + b.w)) + ((c.x + c.y) + (c.z + c.w)) +
+                      ((e.x + e.y) + (e.z + e.w));
+    return 1.0f / sqrtf(tot / (float)d + P.dm.eps);
 }
 
 // ------------------------------------------------------------------ row GEMV
@@ -505,7 +533,7 @@ __device__ __forceinline__ float rms_scale(const Smem& sm, int d, float eps) {
 // unit sums go to work[row * gs + slice]; the caller sums the slices after a CTA barrier.
 template <int NCH, int GM>
 __device__ __forceinline__ void gemv_rows(const Params& P, const Smem& sm, const unsigned long long* ctl, int nrows,
-                                          const __nv_bfloat16* gain, float scale, Ring& rg, bool& ok, Tracer& tr) {
+                                          float scale, Ring& rg, bool& ok, Tracer& tr) {
     const int d = P.dm.d;
     const int gs = P.sh.gs, gr = P.sh.gr;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -521,7 +549,7 @@ __device__ __forceinline__ void gemv_rows(const Params& P, const Smem& sm, const
         const int k = sl * slen + (lane + 32 * i) * 8;
         const float4 a = *reinterpret_cast<const float4*>(sm.x + k);
         const float4 b = *reinterpret_cast<const float4*>(sm.x + k + 4);
-        const uint4 g = __ldg(reinterpret_cast<const uint4*>(gain + k));
+        const uint4 g = lds128(sm.gain + k);
         xr[i][0] = (a.x * scale) * bf_lo(g.x), xr[i][1] = (a.y * scale) * bf_hi(g.x);
         xr[i][2] = (a.z * scale) * bf_lo(g.y), xr[i][3] = (a.w * scale) * bf_hi(g.y);
         xr[i][4] = (b.x * scale) * bf_lo(g.z), xr[i][5] = (b.y * scale) * bf_hi(g.z);
@@ -529,17 +557,41 @@ __device__ __forceinline__ void gemv_rows(const Params& P, const Smem& sm, const
     }
     const int loff = sl * slen * 2 + lane * 16;  // this lane's first chunk in a row; then +512 B each
 
-    constexpr int SG = 4 / GM;  // stages per reduction group
+    // Stages are taken in batches of SB = SG / 2 (two stages when GM == 1): the batch's
+    // stages are awaited together and their dot products formed together, so the fixed
+    // latency of a stage hand-off (mbarrier wait, loads, FMA chain, release) is paid once per
+    // batch and the batch's units give each warp independent chains to interleave.
+    // The lane partials of four units (SG = 4 / GM stages) are then reduced together: value i
+    // belongs to stage j0 + i / GM and row rw + (i % GM) * rstep. After the last stage of the
+    // phase the group may be short; its missing values are zero and are not written.
+    constexpr int SG = 4 / GM;
+    constexpr int SB = SG >= 2 ? 2 : 1;
     for (int j0 = 0; j0 < nst; j0 += SG) {
         float v[4];
 #pragma unroll
-        for (int s = 0; s < SG; ++s) {
-            const int j = j0 + s;
+        for (int i = 0; i < 4; ++i) v[i] = 0.f;
 #pragma unroll
-            for (int u = 0; u < GM; ++u) v[s * GM + u] = 0.f;
-            if (j < nst) {
-                if (ok && wait_full(sm, rg, P, ctl, tr.waited)) {
-                    const uint8_t* st = sm.ring + (size_t)rg.slot * kStageBytes;
+        for (int b0 = 0; b0 < SG; b0 += SB) {
+            Ring rgs[SB];
+            bool have[SB];
+            bool all = true;
+#pragma unroll
+            for (int q = 0; q < SB; ++q) {
+                const int j = j0 + b0 + q;
+                have[q] = j < nst;
+                rgs[q] = rg;
+                if (have[q]) {
+                    rg.advance(P.ns);
+                    if (ok && wait_full(sm, rgs[q], P, ctl, tr.waited)) tr.stage_ready(j, nst);
+                    else all = false;
+                }
+            }
+            if (!all) ok = false;
+#pragma unroll
+            for (int q = 0; q < SB; ++q) {
+                const int j = j0 + b0 + q;
+                if (have[q] && ok) {
+                    const uint8_t* st = sm.ring + (size_t)rgs[q].slot * kStageBytes;
                     const int nr = min(gr, nrows - j * gr);
 #pragma unroll
                     for (int u = 0; u < GM; ++u) {
@@ -559,50 +611,48 @@ __device__ __forceinline__ void gemv_rows(const Params& P, const Smem& sm, const
                                 a2 = fmaf(bf_lo(w.w), xr[i][6], a2);
                                 a3 = fmaf(bf_hi(w.w), xr[i][7], a3);
                             }
-                            v[s * GM + u] = (a0 + a1) + (a2 + a3);
+                            v[(b0 + q) * GM + u] = (a0 + a1) + (a2 + a3);
                         }
                     }
-                    release(sm, rg);
-                } else {
-                    ok = false;
                 }
-                rg.advance(P.ns);
             }
-        }
-        // value i (stage j0 + i / GM, row rw + (i % GM) * rstep) ends in lanes 8i..8i+7
-        const bool b4 = lane & 16, b3 = lane & 8;
-        float w2[2];
 #pragma unroll
-        for (int k = 0; k < 2; ++k)
-            w2[k] = (b4 ? v[2 + k] : v[k]) + __shfl_xor_sync(0xffffffffu, b4 ? v[k] : v[2 + k], 16);
-        float z = (b3 ? w2[1] : w2[0]) + __shfl_xor_sync(0xffffffffu, b3 ? w2[0] : w2[1], 8);
+            for (int q = 0; q < SB; ++q)
+                if (have[q] && ok) release(sm, rgs[q]);
+        }
+        // exchange levels 16 and 8 halve the values a lane holds; levels 4, 2, 1 finish the
+        // 32-lane sums: value i ends in lanes 8i..8i+7
+        const bool b4 = lane & 16, b3 = lane & 8;
+        const float w0 = (b4 ? v[2] : v[0]) + __shfl_xor_sync(0xffffffffu, b4 ? v[0] : v[2], 16);
+        const float w1 = (b4 ? v[3] : v[1]) + __shfl_xor_sync(0xffffffffu, b4 ? v[1] : v[3], 16);
+        float z = (b3 ? w1 : w0) + __shfl_xor_sync(0xffffffffu, b3 ? w0 : w1, 8);
         z += __shfl_xor_sync(0xffffffffu, z, 4);
         z += __shfl_xor_sync(0xffffffffu, z, 2);
         z += __shfl_xor_sync(0xffffffffu, z, 1);
         if ((lane & 7) == 0 && ok) {
             const int i = lane >> 3;
-            const int j = j0 + i / GM, row = rw + (i % GM) * rstep;
-            if (j < nst && row < min(gr, nrows - j * gr)) sm.work[(j * gr + row) * gs + sl] = z;
+            const int js = j0 + i / GM, row = rw + (i % GM) * rstep;
+            if (js < nst && row < min(gr, nrows - js * gr)) sm.work[(js * gr + row) * gs + sl] = z;
         }
     }
 }
 
 // Dispatch on the chunks per lane and units per warp (fixed per model).
 __device__ __forceinline__ void run_rows(const Params& P, const Smem& sm, const unsigned long long* ctl, int nrows,
-                                         const __nv_bfloat16* gain, float scale, Ring& rg, bool& ok, Tracer& tr) {
+                                         float scale, Ring& rg, bool& ok, Tracer& tr) {
     const int nch = P.dm.d / P.sh.gs / 256;
     const int gm = P.sh.gm;
     if (gm == 1) {
         switch (nch) {
-            case 1: gemv_rows<1, 1>(P, sm, ctl, nrows, gain, scale, rg, ok, tr); break;
-            case 2: gemv_rows<2, 1>(P, sm, ctl, nrows, gain, scale, rg, ok, tr); break;
-            case 3: gemv_rows<3, 1>(P, sm, ctl, nrows, gain, scale, rg, ok, tr); break;
-            default: gemv_rows<4, 1>(P, sm, ctl, nrows, gain, scale, rg, ok, tr); break;
+            case 1: gemv_rows<1, 1>(P, sm, ctl, nrows, scale, rg, ok, tr); break;
+            case 2: gemv_rows<2, 1>(P, sm, ctl, nrows, scale, rg, ok, tr); break;
+            case 3: gemv_rows<3, 1>(P, sm, ctl, nrows, scale, rg, ok, tr); break;
+            default: gemv_rows<4, 1>(P, sm, ctl, nrows, scale, rg, ok, tr); break;
         }
     } else if (gm == 2) {
-        gemv_rows<2, 2>(P, sm, ctl, nrows, gain, scale, rg, ok, tr);
+        gemv_rows<2, 2>(P, sm, ctl, nrows, scale, rg, ok, tr);
     } else {
-        gemv_rows<1, 4>(P, sm, ctl, nrows, gain, scale, rg, ok, tr);
+        gemv_rows<1, 4>(P, sm, ctl, nrows, scale, rg, ok, tr);
     }
 }
 
@@ -637,6 +687,7 @@ __device__ __forceinline__ void gemv_splitk(const Params& P, const Smem& sm, con
         for (int e = 0; e < 8; ++e) acc[c][e] = 0.f;
     for (int j = 0; j < nst; ++j) {
         if (ok && wait_full(sm, rg, P, ctl, tr.waited)) {
+            tr.stage_ready(j, nst);
             const uint8_t* st = sm.ring + (size_t)rg.slot * kStageBytes;
             const int nr = min(kr, nrows - j * kr);
             if (active) {
@@ -807,6 +858,7 @@ __device__ __forceinline__ void run_attention(const Params& P, const Smem& sm, c
         for (int js = 0; js < nks; ++js) {
             float* sp = spart + (size_t)(js & 1) * NQ * GM * PPS;
             if (ok && wait_full(sm, rg, P, ctl, tr.waited)) {
+                if (kb == 0 && js == 0) tr.mark(6);
                 const uint8_t* st = sm.ring + (size_t)rg.slot * kStageBytes;
                 const int nv = min(PPS, n - js * PPS);
                 // chunk c of this thread's quarter is taken in a rotated order (c + jpos) & 3,
@@ -924,6 +976,7 @@ __device__ __forceinline__ void run_attention(const Params& P, const Smem& sm, c
         // ---- V stages
         for (int js = 0; js < nks; ++js) {
             if (ok && wait_full(sm, rg, P, ctl, tr.waited)) {
+                if (last && js == nks - 1) tr.mark(7);
                 const uint8_t* st = sm.ring + (size_t)rg.slot * kStageBytes;
                 const int nv = min(PPS, n - js * PPS);
                 for (int j = pg; j < nv; j += NPG) {
@@ -987,19 +1040,19 @@ __device__ __forceinline__ void run_attention(const Params& P, const Smem& sm, c
     }
 }
 
-// Output projection: combine the attention records of every piece of this CTA's kv head
-// for its own output dims (pieces in order: max-rescaled sums), then multiply them by the
-// matching transposed output-projection rows and add the partial d-vector into `dst`.
+// Output-projection inputs: combine the attention records of every piece of this CTA's kv
+// head for its own output dims (pieces in order: max-rescaled sums) into sm.hin. Returns the
+// number of dims (rows of the transposed output projection this CTA multiplies).
 template <int HD>
-__device__ __forceinline__ void run_oproj(const Params& P, const Smem& sm, const unsigned long long* ctl, int t, int l,
-                                          float* dst, Ring& rg, bool& ok, Tracer& tr) {
+__device__ __forceinline__ int oproj_inputs(const Params& P, const Smem& sm, const unsigned long long* ctl, int t, int l,
+                                            bool& ok, Tracer& tr) {
     const Dims& dm = P.dm;
     const Geo& g = *sm.geo;
     const int r = dm.r, A = P.pieces;
     const int cc = r * HD;
     const int c0 = g.o0 - g.grp * cc, c1 = g.o1 - g.grp * cc;  // dims within the kv head's heads
     const int ncol = c1 - c0;
-    if (ncol <= 0) return;  // more pieces than output dims: this CTA has none (uniform)
+    if (ncol <= 0) return 0;  // more pieces than output dims: this CTA has none (uniform)
     const int h0 = c0 / HD, h1 = (c1 - 1) / HD, nh = h1 - h0 + 1;
     const int W = 2 * nh + ncol;  // words per piece: (max, sum) per head, then acc per dim
     const uint32_t tag = qkv_tag(P, t, l) + 1u;
@@ -1037,10 +1090,88 @@ __device__ __forceinline__ void run_oproj(const Params& P, const Smem& sm, const
         sm.hin[j] = o / L;
     }
     consumer_sync();
-    run_splitk(P, sm, ctl, ncol, sm.hin, dst, rg, ok, tr);
+    return ncol;
 }
 
 // ------------------------------------------------------------------ producer
+
+// Walks this CTA's stages in consumption order: per step, per layer the Q/K/V rows, the
+// attention piece (per softmax block its K stages, then its V stages), the output-projection
+// rows, the gate/up rows, the down-projection rows; then the LM-head rows at steps that run
+// the head. Sub-phase `sub` of a layer: 0 Q/K/V, 1 .. 2 * nblk attention (block (sub - 1) / 2,
+// K for odd sub, V for even), then output projection, gate/up, down, and after the last layer
+// the LM head.
+struct Walk {
+    int t = 0, l = 0, sub = 0, j = 0;
+    int pc_t = -1;
+    Piece pc;
+    bool done = false;
+
+    // The current sub-phase's rows: base, bytes per row, rows, rows per stage, and the first
+    // cache position (-1 for weights).
+    __device__ void desc(const Params& P, const Geo& g, const uint8_t*& base, size_t& rowb, int& nrows, int& per,
+                         int& pos) {
+        const Dims& dm = P.dm;
+        const size_t wrow = (size_t)dm.d * 2;
+        const uint8_t* lb = P.arena + P.lay.layer0 + (size_t)l * P.lay.layer_stride;
+        const int natt = g.grp < 0 ? 0 : 2 * pc.nblk;
+        pos = -1;
+        rowb = wrow;
+        if (sub == 0) {
+            base = lb + P.lay.l_wqkv + (size_t)g.q0 * wrow, nrows = g.q1 - g.q0, per = P.sh.gr;
+        } else if (sub <= natt) {
+            const int kb = (sub - 1) / 2;
+            const int s0 = pc.a + kb * P.blk;
+            const size_t head = ((size_t)l * dm.Hkv + g.grp) * dm.S;
+            rowb = (size_t)dm.hd * 2;
+            base = P.arena + ((sub & 1) ? P.lay.kcache : P.lay.vcache) + (head + s0) * rowb;
+            nrows = block_len(P, pc, kb), per = kStageBytes / (int)rowb, pos = s0;
+        } else if (sub == natt + 1) {
+            base = lb + P.lay.l_wot + (size_t)g.o0 * wrow, nrows = g.o1 - g.o0, per = P.sh.kr;
+        } else if (sub == natt + 2) {
+            base = lb + P.lay.l_wgu + (size_t)2 * g.u0 * wrow, nrows = 2 * (g.u1 - g.u0), per = P.sh.gr;
+        } else if (sub == natt + 3) {
+            base = lb + P.lay.l_wdt + (size_t)g.u0 * wrow, nrows = g.u1 - g.u0, per = P.sh.kr;
+        } else {
+            base = P.arena + P.lay.lm_head + (size_t)g.v0 * wrow, nrows = g.v1 - g.v0, per = P.sh.gr;
+        }
+    }
+    __device__ int nsubs(const Params& P, const Geo& g) const {
+        const int natt = g.grp < 0 ? 0 : 2 * pc.nblk;
+        return natt + 4 + (l == P.dm.L - 1 && step_has_head(P, t) ? 1 : 0);
+    }
+    // The next stage: source, bytes, and the last cache position it reads (-1 for weights).
+    // Returns false when the launch's stages are exhausted.
+    __device__ bool next(const Params& P, const Geo& g, const uint8_t*& src, uint32_t& bytes, int& kv_last) {
+        for (;;) {
+            if (done) return false;
+            if (pc_t != t) {
+                pc = piece_geo(P, g.piece, P.pos0 + t);
+                pc_t = t;
+            }
+            const uint8_t* base;
+            size_t rowb;
+            int nrows, per, pos;
+            desc(P, g, base, rowb, nrows, per, pos);
+            if (j * per < nrows) {
+                const int n = min(per, nrows - j * per);
+                src = base + (size_t)j * per * rowb;
+                bytes = (uint32_t)(n * rowb);
+                kv_last = pos < 0 ? -1 : pos + j * per + n - 1;
+                ++j;
+                return true;
+            }
+            j = 0;
+            if (++sub >= nsubs(P, g)) {
+                sub = 0;
+                if (++l == P.dm.L) {
+                    l = 0;
+                    if (++t == P.steps) done = true;
+                }
+            }
+        }
+    }
+};
 
 struct Producer {
     const Params& P;
@@ -1067,12 +1198,11 @@ struct Producer {
         const long long c0 = clock64();
         Deadline dl;
         for (;;) {
-            if (mbar_wait_hint(a, par)) {
-                wait_slot += (unsigned long long)(clock64() - c0);
-                return true;
-            }
+            if (mbar_wait_hint(a, par)) break;
             if (!dl.alive(ctl, P.timeout_ns, where_code(kWhereEmpty, slot))) return false;
         }
+        wait_slot += (unsigned long long)(clock64() - c0);
+        return true;
     }
 
     // Wait until at least `need` syncs of this launch have completed, then order the
@@ -1091,7 +1221,13 @@ struct Producer {
         return true;
     }
 
-    __device__ bool issue(const void* src, uint32_t bytes) {
+    // Stage k into its ring slot. A cache row written earlier in this launch (at step s) is
+    // read only after the last sync of step s, which orders that step's cache writes.
+    __device__ bool issue(const uint8_t* src, uint32_t bytes, int kv_last) {
+        if (kv_last >= P.pos0) {
+            const int s = kv_last - P.pos0;
+            if (!wait_syncs(syncs_before_step(P.dm.L, s + 1, P.n_pending, P.dump != 0))) return false;
+        }
         if (!wait_empty()) return false;
         const uint32_t fb = smem_u32(&sm.full[slot]);
         mbar_expect_tx(fb, bytes);
@@ -1104,58 +1240,15 @@ struct Producer {
         return true;
     }
 
-    // `nrows` rows of `rowbytes` from `src`, `per` rows per stage.
-    __device__ bool rows(const uint8_t* src, int nrows, int per, size_t rowbytes) {
-        for (int j = 0; j < nrows; j += per) {
-            const int n = min(per, nrows - j);
-            if (!issue(src + (size_t)j * rowbytes, (uint32_t)(n * rowbytes))) return false;
-        }
-        return true;
-    }
-
-    // The cached K and V rows of this CTA's attention piece at step t, layer l: per block,
-    // its K stages, then its V stages. A row written earlier in this launch (at step s) is
-    // read only after the last sync of step s, which orders that step's cache writes.
-    __device__ bool kv(const Geo& g, int t, int l) {
-        const Dims& dm = P.dm;
-        const int hd = dm.hd, pps = kStageBytes / (2 * hd);
-        const Piece pc = piece_geo(P, g.piece, P.pos0 + t);
-        const size_t head = ((size_t)l * dm.Hkv + g.grp) * dm.S;
-        const uint8_t* kb = P.arena + P.lay.kcache + head * hd * 2;
-        const uint8_t* vb = P.arena + P.lay.vcache + head * hd * 2;
-        for (int b = 0; b < pc.nblk; ++b) {
-            const int s0 = pc.a + b * P.blk, n = block_len(P, pc, b);
-            if (n > 0 && s0 + n - 1 >= P.pos0) {
-                const int s = s0 + n - 1 - P.pos0;  // step that appended the block's last row
-                if (!wait_syncs(syncs_before_step(dm.L, s + 1, P.n_pending, P.dump != 0))) return false;
-            }
-            for (int which = 0; which < 2; ++which) {
-                const uint8_t* src = (which ? vb : kb) + (size_t)s0 * hd * 2;
-                if (!rows(src, n, pps, (size_t)hd * 2)) return false;
-            }
-        }
-        return true;
-    }
-
     __device__ void run() {
         const long long c_start = clock64();
-        const Dims& dm = P.dm;
         const Geo g = *sm.geo;
-        const size_t rowb = (size_t)dm.d * 2;
-        const uint8_t* l0 = P.arena + P.lay.layer0;
+        Walk ring;
+        const uint8_t* src;
+        uint32_t bytes;
+        int kv_last;
         bool ok = true;
-        for (int t = 0; t < P.steps && ok; ++t) {
-            for (int l = 0; l < dm.L && ok; ++l) {
-                const uint8_t* lb = l0 + (size_t)l * P.lay.layer_stride;
-                ok = rows(lb + P.lay.l_wqkv + (size_t)g.q0 * rowb, g.q1 - g.q0, P.sh.gr, rowb) &&
-                     (g.grp < 0 || kv(g, t, l)) &&
-                     rows(lb + P.lay.l_wot + (size_t)g.o0 * rowb, g.o1 - g.o0, P.sh.kr, rowb) &&
-                     rows(lb + P.lay.l_wgu + (size_t)2 * g.u0 * rowb, 2 * (g.u1 - g.u0), P.sh.gr, rowb) &&
-                     rows(lb + P.lay.l_wdt + (size_t)g.u0 * rowb, g.u1 - g.u0, P.sh.kr, rowb);
-            }
-            if (ok && step_has_head(P, t))
-                ok = rows(P.arena + P.lay.lm_head + (size_t)g.v0 * rowb, g.v1 - g.v0, P.sh.gr, rowb);
-        }
+        while (ok && ring.next(P, g, src, bytes, kv_last)) ok = issue(src, bytes, kv_last);
         // Let every copy already issued land before the CTA exits: when the consumers have
         // stopped early (a refused token, a wait that gave up) nobody else waits for them.
         // On a normal run these stages were consumed already and each test passes at once.
@@ -1286,110 +1379,83 @@ __global__ void __launch_bounds__(kThreads, 1) monokernel(const __grid_constant_
         }
         consumer_sync();
 
-        for (int l = 0; l < dm.L && ok; ++l) {
+        // The step's phases in order: per layer Q/K/V, attention, output projection, gate/up,
+        // down; then the LM head if this step picks a token. One loop with one call site per
+        // phase kind keeps a single copy of each phase's code in the kernel (the executed
+        // code then stays in the instruction cache across layers).
+        const int nphase = 5 * dm.L + (step_has_head(P, t) ? 1 : 0);
+        for (int q = 0; q < nphase && ok; ++q) {
+            const int l = q / 5 < dm.L ? q / 5 : dm.L - 1;
+            const int ph = q / 5 < dm.L ? q % 5 : kLM;
             const uint8_t* lb = l0 + (size_t)l * P.lay.layer_stride;
-            const uint32_t tag = qkv_tag(P, t, l);
-            // ---- Q/K/V
-            tr.begin((t << 16) | (l << 4) | kQKV);
-            if (l > 0) {
-                ok = sync_wait(sm, P, ctl, k - 1, ok);
-                if (!ok) break;
-                fold_delta(sm, P, k - 1);
-            }
-            tr.mark(2);
-            {
-                const float s = rms_scale(sm, dm.d, dm.eps);
-                run_rows(P, sm, ctl, g.q1 - g.q0, reinterpret_cast<const __nv_bfloat16*>(lb + P.lay.l_attn_norm), s,
-                         rg, ok, tr);
-                ok = consumer_sync_and(ok);
-                tr.mark(3);
-                if (ok && g.grp >= 0) qkv_epilogue(P, sm, g, l, p, tag);
-            }
-            tr.end();
-            if (!ok) break;
-            // ---- attention piece
-            tr.begin((t << 16) | (l << 4) | kATT);
-            if (g.grp >= 0) run_attention<HD, GM>(P, sm, ctl, t, l, rg, ok, tr);
-            ok = consumer_sync_and(ok);
-            tr.end();
-            if (!ok) break;
-            // ---- output projection (split-K) -> sync k
-            tr.begin((t << 16) | (l << 4) | kO);
-            float* dO = delta + (size_t)(k % 3) * dm.d;
-            if (g.grp >= 0) run_oproj<HD>(P, sm, ctl, t, l, dO, rg, ok, tr);
-            tr.mark(3);
-            ok = consumer_sync_and(ok);
-            if (ok) sync_arrive(ctl);
-            ++k;
-            tr.end();
-            if (!ok) break;
-            // ---- gate/up with SwiGLU
-            tr.begin((t << 16) | (l << 4) | kGU);
-            ok = sync_wait(sm, P, ctl, k - 1, ok);
-            if (!ok) break;
-            fold_delta(sm, P, k - 1);
-            tr.mark(2);
-            {
-                const float s = rms_scale(sm, dm.d, dm.eps);
-                run_rows(P, sm, ctl, 2 * (g.u1 - g.u0), reinterpret_cast<const __nv_bfloat16*>(lb + P.lay.l_ffn_norm), s,
-                         rg, ok, tr);
-                consumer_sync();
-                for (int j = tid; j < g.u1 - g.u0; j += kConsumerThreads) {
-                    const float gt = row_value(sm, P.sh.gs, 2 * j), up = row_value(sm, P.sh.gs, 2 * j + 1);
-                    sm.hin[j] = gt / (1.0f + expf(-gt)) * up;
+            tr.begin((t << 16) | (l << 4) | ph);
+            if (ph == kQKV || ph == kGU || ph == kLM) {
+                // ---- row GEMV: Q/K/V, gate/up or LM head over the normalised residual
+                const uint8_t* gain = ph == kQKV ? lb + P.lay.l_attn_norm
+                                      : ph == kGU ? lb + P.lay.l_ffn_norm : P.arena + P.lay.final_norm;
+                prefetch_gain(sm, reinterpret_cast<const __nv_bfloat16*>(gain), dm.d);
+                const bool after_sync = !(ph == kQKV && l == 0);  // the first Q/K/V reads the embedding
+                if (after_sync) {
+                    ok = sync_wait(sm, P, ctl, k - 1, ok);
+                    if (!ok) break;
                 }
+                const float s = fold_norm(sm, P, after_sync ? k - 1 : -1);
+                tr.mark(2);
+                const int nrows = ph == kQKV ? g.q1 - g.q0 : ph == kGU ? 2 * (g.u1 - g.u0) : g.v1 - g.v0;
+                run_rows(P, sm, ctl, nrows, s, rg, ok, tr);
                 ok = consumer_sync_and(ok);
-            }
-            tr.mark(3);
-            tr.end();
-            if (!ok) break;
-            // ---- down projection (split-K) -> sync k
-            tr.begin((t << 16) | (l << 4) | kD);
-            float* dD = delta + (size_t)(k % 3) * dm.d;
-            run_splitk(P, sm, ctl, g.u1 - g.u0, sm.hin, dD, rg, ok, tr);
-            tr.mark(3);
-            ok = consumer_sync_and(ok);
-            if (ok) sync_arrive(ctl);
-            ++k;
-            tr.end();
-        }
-        if (!ok) break;
-        // ---- LM head and argmax -> sync k
-        if (step_has_head(P, t)) {
-            tr.begin((t << 16) | kLM);
-            ok = sync_wait(sm, P, ctl, k - 1, ok);
-            if (!ok) break;
-            fold_delta(sm, P, k - 1);
-            tr.mark(2);
-            const float s = rms_scale(sm, dm.d, dm.eps);
-            run_rows(P, sm, ctl, g.v1 - g.v0, reinterpret_cast<const __nv_bfloat16*>(P.arena + P.lay.final_norm), s, rg, ok,
-                     tr);
-            consumer_sync();
-            unsigned long long best = 0ull;
-            for (int i = tid; i < g.v1 - g.v0; i += kConsumerThreads) {
-                const float y = row_value(sm, P.sh.gs, i);
-                if (P.dump) __stcg(P.logits_out + (size_t)t * dm.V + g.v0 + i, y);
-                const unsigned long long key = argmax_key(y, g.v0 + i);
-                best = key > best ? key : best;
-            }
+                if (ph == kQKV) {
+                    tr.mark(3);
+                    if (ok && g.grp >= 0) qkv_epilogue(P, sm, g, l, p, qkv_tag(P, t, l));
+                } else if (ph == kGU) {
+                    for (int j = tid; j < g.u1 - g.u0; j += kConsumerThreads) {
+                        const float gt = row_value(sm, P.sh.gs, 2 * j), up = row_value(sm, P.sh.gs, 2 * j + 1);
+                        sm.hin[j] = gt / (1.0f + expf(-gt)) * up;
+                    }
+                    ok = consumer_sync_and(ok);
+                    tr.mark(3);
+                } else {
+                    unsigned long long best = 0ull;
+                    for (int i = tid; i < g.v1 - g.v0; i += kConsumerThreads) {
+                        const float y = row_value(sm, P.sh.gs, i);
+                        if (P.dump) __stcg(P.logits_out + (size_t)t * dm.V + g.v0 + i, y);
+                        const unsigned long long key = argmax_key(y, g.v0 + i);
+                        best = key > best ? key : best;
+                    }
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                const unsigned long long other = __shfl_xor_sync(0xffffffffu, best, o);
-                best = other > best ? other : best;
-            }
-            if ((tid & 31) == 0) reinterpret_cast<unsigned long long*>(sm.red)[tid >> 5] = best;
-            ok = consumer_sync_and(ok);
-            if (tid == 0 && ok) {
-                unsigned long long b = 0ull;
-                for (int w = 0; w < kConsumerWarps; ++w) {
-                    const unsigned long long v = reinterpret_cast<unsigned long long*>(sm.red)[w];
-                    b = v > b ? v : b;
+                    for (int o = 16; o > 0; o >>= 1) {
+                        const unsigned long long other = __shfl_xor_sync(0xffffffffu, best, o);
+                        best = other > best ? other : best;
+                    }
+                    if ((tid & 31) == 0) reinterpret_cast<unsigned long long*>(sm.red)[tid >> 5] = best;
+                    ok = consumer_sync_and(ok);
+                    if (tid == 0 && ok) {
+                        unsigned long long b = 0ull;
+                        for (int w = 0; w < kConsumerWarps; ++w) {
+                            const unsigned long long v = reinterpret_cast<unsigned long long*>(sm.red)[w];
+                            b = v > b ? v : b;
+                        }
+                        red_max_u64(ctl + kCtlArgmax + 16 * (t % 3), b);
+                    }
+                    tr.mark(3);
+                    if (ok) sync_arrive(ctl);  // -> sync k: the step's argmax is complete
+                    ++k;
                 }
-                atomicMax(ctl + kCtlArgmax + 16 * (t % 3), b);
+            } else if (ph == kATT) {
+                // ---- attention piece
+                if (g.grp >= 0) run_attention<HD, GM>(P, sm, ctl, t, l, rg, ok, tr);
+                ok = consumer_sync_and(ok);
+            } else {
+                // ---- split-K output projection or down projection -> sync k
+                tr.mark(2);
+                int nrows = g.u1 - g.u0;  // down: this CTA's hidden units (sm.hin, from gate/up)
+                if (ph == kO) nrows = g.grp >= 0 ? oproj_inputs<HD>(P, sm, ctl, t, l, ok, tr) : 0;
+                run_splitk(P, sm, ctl, nrows, sm.hin, delta + (size_t)(k % 3) * dm.d, rg, ok, tr);
+                tr.mark(3);
+                ok = consumer_sync_and(ok);
+                if (ok) sync_arrive(ctl);
+                ++k;
             }
-            tr.mark(3);
-            if (ok) sync_arrive(ctl);
-            ++k;
             tr.end();
         }
     }

@@ -137,7 +137,8 @@ struct Params {
 
 // Trace row layout (SM clock cycles), one row per phase of a traced CTA, in phase order:
 // [phase id (step << 16 | layer << 4 | phase), begin, inputs ready, compute done, end,
-//  cycles waiting for weight / KV stages, 0, 0]. The last row of a traced CTA holds the
+//  cycles waiting for weight / KV stages, first stage ready, last stage ready] (the last two
+//  are 0 in a phase without stages). The last row of a traced CTA holds the
 // producer warp's [cycles waiting for a free stage, cycles waiting for KV rows written this
 // launch, stages issued, total cycles].
 constexpr int kTraceWords = 8;

@@ -24,11 +24,13 @@ ATOL = 2e-2
 REL_L2 = 1e-3
 MARGIN = 5e-2
 # Two launches of the same request differ only in the order of the fp32 atomic additions
-# that sum the split-K output and down projections (a few ulps per layer): their logits
-# agree far inside the parity tolerance, and their tokens agree except where the top two
-# logits are closer than that noise.
-RUN_REL_L2 = 1e-5
-RUN_MARGIN = 1e-3
+# that sum the split-K output and down projections (a few ulps per layer). Where a model
+# writes its own KV cache those ulps now and then round a K or V element to the
+# neighbouring bf16 value, so two runs are two equally valid fp32 results: their logits must
+# agree within the parity tolerance, and their tokens wherever the top two logits are
+# further apart than those differences can reach.
+RUN_REL_L2 = REL_L2
+RUN_MARGIN = 2e-2
 
 
 def oracle_threads() -> int:
@@ -107,7 +109,9 @@ def compare_gpu_runs(toks_a, toks_b, logits_a, what: str = "", logits_b=None):
     for i in range(len(toks_a)):
         if logits_b is not None:
             rel = float(rel_l2(logits_b[i:i + 1], logits_a[i:i + 1])[0])
-            assert rel <= RUN_REL_L2, "%s: step %d runs differ by rel-L2 %.3g" % (what, i, rel)
+            mx = float(np.abs(logits_b[i].astype(np.float64) - logits_a[i]).max())
+            assert rel <= RUN_REL_L2 and mx <= ATOL, "%s: step %d runs differ by rel-L2 %.3g, max|d| %.3g" % (
+                what, i, rel, mx)
         if int(toks_a[i]) != int(toks_b[i]):
             m = margin(logits_a[i])
             assert m < RUN_MARGIN, "%s: runs diverge at step %d with margin %.3g" % (what, i, m)
