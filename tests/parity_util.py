@@ -54,18 +54,25 @@ def rel_bound_from_exact(oracle_logits: np.ndarray, exact_logits: np.ndarray) ->
     return np.maximum(REL_L2, 2.0 * rel_l2(oracle_logits, exact_logits))
 
 
-def check_logits(gpu: np.ndarray, ref: np.ndarray, what: str = "", rel_bound=None):
+def atol_bound_from_exact(oracle_logits: np.ndarray, exact_logits: np.ndarray) -> np.ndarray:
+    """Per-step max|delta| bound: max(2e-2, 2 * the oracle's own max|delta| against the exact forward)."""
+    d = np.abs(np.asarray(oracle_logits, np.float64) - np.asarray(exact_logits, np.float64)).max(axis=1)
+    return np.maximum(ATOL, 2.0 * d)
+
+
+def check_logits(gpu: np.ndarray, ref: np.ndarray, what: str = "", rel_bound=None, atol_bound=None):
     """gpu, ref: [n][V]. Asserts the tolerance at every row; returns (max abs, max rel-L2).
-    rel_bound: per-row rel-L2 bounds (default 1e-3 everywhere)."""
+    rel_bound / atol_bound: per-row bounds (default 1e-3 and 2e-2 everywhere)."""
     assert gpu.shape == ref.shape, (gpu.shape, ref.shape)
     assert np.all(np.isfinite(gpu)), "%s: non-finite GPU logits" % what
     d = np.abs(gpu.astype(np.float64) - ref.astype(np.float64))
     mx = d.max(axis=1)
     rel = rel_l2(gpu, ref)
     bound = np.full(len(rel), REL_L2) if rel_bound is None else np.asarray(rel_bound)
-    bad = np.nonzero((mx > ATOL) | (rel > bound))[0]
-    assert bad.size == 0, "%s: step %d max|d| %.3g rel-L2 %.3g (bound %.3g)" % (
-        what, bad[0], mx[bad[0]], rel[bad[0]], bound[bad[0]])
+    abound = np.full(len(rel), ATOL) if atol_bound is None else np.asarray(atol_bound)
+    bad = np.nonzero((mx > abound) | (rel > bound))[0]
+    assert bad.size == 0, "%s: step %d max|d| %.3g rel-L2 %.3g (bounds %.3g, %.3g)" % (
+        what, bad[0], mx[bad[0]], rel[bad[0]], abound[bad[0]], bound[bad[0]])
     return float(mx.max()), float(rel.max())
 
 

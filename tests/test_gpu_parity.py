@@ -12,8 +12,9 @@ import torch
 import oracle
 from oracle import naive
 import synth
-from tests.parity_util import (check_logits, check_tokens_against_logits, compare_free_run, compare_gpu_runs,
-                               oracle_threads, rel_bound_from_exact)
+from oracle import exact
+from tests.parity_util import (REL_L2, atol_bound_from_exact, check_logits, check_tokens_against_logits,
+                               compare_free_run, compare_gpu_runs, oracle_threads, rel_bound_from_exact, rel_l2)
 
 pytestmark = [pytest.mark.gpu,
               pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA GPU")]
@@ -61,8 +62,10 @@ def test_tiny_forced_logits_every_step(kd):
     dec.sync()
     gpu = lg.cpu().numpy()
     ref = oracle.Oracle(w.dims(), W, capacity=len(toks)).forced(toks, 0)
-    bound = rel_bound_from_exact(ref, naive.causal_forward(w.dims(), W, toks))
-    check_logits(gpu, ref, "tiny forced", bound)
+    ex = naive.causal_forward(w.dims(), W, toks)
+    rb, ab = rel_bound_from_exact(ref, ex), atol_bound_from_exact(ref, ex)
+    check_logits(gpu, ex, "tiny forced vs exact", rb, ab)
+    check_logits(gpu, ref, "tiny forced", rb, ab)
     check_tokens_against_logits(gpu.argmax(axis=1), ref, "tiny forced")
 
 
@@ -83,8 +86,8 @@ def test_tiny_greedy_free_run_and_in_kernel_argmax(kd):
     o = oracle.Oracle(w.dims(), W, capacity=w.capacity)
     otoks, ologits = o.greedy(prompt, 0, w.n_gen)
     seq = np.concatenate([prompt, otoks[:-1]])
-    exact = naive.causal_forward(w.dims(), W, seq)[w.prompt_len - 1:]
-    n = compare_free_run(toks, chosen, otoks, ologits, "tiny greedy", rel_bound_from_exact(ologits, exact))
+    ex_g = naive.causal_forward(w.dims(), W, seq)[w.prompt_len - 1:]
+    n = compare_free_run(toks, chosen, otoks, ologits, "tiny greedy", rel_bound_from_exact(ologits, ex_g))
     assert n >= 1
     # the launch that is benchmarked (no logits) picks the same tokens
     dec.reset(prompt, 0)
@@ -320,8 +323,21 @@ def test_half_billion_forced_and_greedy(kd):
     dec.sync()
     Wh = host(W)
     ref = oracle.Oracle(w.dims(), Wh, capacity=len(toks), n_threads=oracle_threads()).forced(toks, 0)
-    bound = rel_bound_from_exact(ref, naive.causal_forward(w.dims(), Wh, toks))
-    check_logits(lg.cpu().numpy(), ref, "0.5b forced", bound)
+    ex = naive.causal_forward(w.dims(), Wh, toks)
+    gpu = lg.cpu().numpy()
+    # This model writes its own cache, and its logits move by ~4e-3 between rounding the K/V
+    # appends to bf16 and not rounding them: one element that two correct fp32 computations
+    # round to neighbouring bf16 values moves a step by up to ~1e-3. So the GPU is held, against
+    # the exact float64 forward and against the fp32 oracle alike, to the tolerance widened to
+    # twice the oracle's own distance from the exact forward where that is larger.
+    rb, ab = rel_bound_from_exact(ref, ex), atol_bound_from_exact(ref, ex)
+    mx_e, rel_e = check_logits(gpu, ex, "0.5b forced vs exact", rb, ab)
+    mx_o, rel_o = check_logits(gpu, ref, "0.5b forced", rb, ab)
+    o_ex = rel_l2(ref, ex)
+    print("\n0.5b | %d forced steps | GPU vs exact: max|d| %.2e, max rel-L2 %.2e | GPU vs oracle: max|d| %.2e, "
+          "max rel-L2 %.2e, steps above 1e-3: %d | oracle vs exact: max rel-L2 %.2e, steps above 1e-3: %d"
+          % (len(toks), mx_e, rel_e, mx_o, rel_o, int((rel_l2(gpu, ref) > REL_L2).sum()), o_ex.max(),
+             int((o_ex > REL_L2).sum())))
     # free-running greedy decode, in the benchmarked launch configuration
     dec.reset(prompt, 0)
     gt, glg = dec.decode(w.n_gen, logits=True)
@@ -335,21 +351,25 @@ def test_half_billion_forced_and_greedy(kd):
     o = oracle.Oracle(w.dims(), Wh, capacity=w.capacity, n_threads=oracle_threads())
     otoks, ologits = o.greedy(prompt, 0, w.n_gen)
     seq = np.concatenate([prompt, otoks[:-1]])
-    exact = naive.causal_forward(w.dims(), Wh, seq)[w.prompt_len - 1:]
-    compare_free_run(gt, chosen, otoks, ologits, "0.5b greedy", rel_bound_from_exact(ologits, exact))
+    ex_g = naive.causal_forward(w.dims(), Wh, seq)[w.prompt_len - 1:]
+    compare_free_run(gt, chosen, otoks, ologits, "0.5b greedy", rel_bound_from_exact(ologits, ex_g))
 
 
 # ------------------------------------------------------------------ large workloads
 
 @pytest.mark.parametrize("name", ["2b-4k", "2b-32k", "8b-4k"])
 def test_full_size_workload(kd, name):
-    """The full benchmarked decode (every token of the workload), checked three ways:
-    * the first 64 steps against the oracle in follow mode: the oracle is fed the GPU's own
-      token history (the start token, then the GPU's tokens), so the two never diverge, and
-      at every one of the 64 steps the logits must be within the tolerance and the GPU token
-      must be the oracle's argmax wherever the oracle's top-1/top-2 margin exceeds 5e-2 (which
-      also makes a free-running oracle agree token for token up to its first step below
-      that margin);
+    """The full benchmarked decode (every token of the workload), checked four ways:
+    * the first 64 steps in follow mode: the GPU's own token history (the start token, then
+      the GPU's tokens) is fed to the oracle and to the exact float64 forward (oracle.exact),
+      so no trajectory diverges; at every one of the 64 steps the GPU logits must be within
+      the tolerance (max|d| <= 2e-2, rel-L2 <= 1e-3) of the exact forward;
+    * at those steps within the tolerance of the oracle too, the bound widened to twice the
+      oracle's own error against the exact forward where that error is larger (the fp32
+      oracle sums 4096-14336-term rows in ascending order and at some 8B steps is ~3e-3 from
+      the exact result), and the GPU token is the oracle's argmax wherever the oracle's
+      top-1/top-2 margin exceeds 5e-2 (which also makes a free-running oracle agree token for
+      token up to its first step below that margin);
     * every step's token equals the argmax of that step's dumped logits;
     * the launch without the logits dump agrees with the dumped one."""
     n_check = 64
@@ -372,13 +392,23 @@ def test_full_size_workload(kd, name):
     assert np.all(np.isfinite(lg))
     assert np.array_equal(toks_d, lg.argmax(axis=1))
     compare_gpu_runs(toks_d, toks, lg, name + " no-dump")
+    del dec
+    torch.cuda.empty_cache()
+    fed = np.concatenate([start, toks_d[:n_check - 1]]).astype(np.int32)
+    ex = exact.causal_forward(w.dims(), W, fed, pos0=w.kv_len, kv_prefix=(K, V), device="cuda")
     Wh = host(W)
-    del W, dec
+    del W
     torch.cuda.empty_cache()
     o = oracle.Oracle(w.dims(), Wh, capacity=w.kv_len + n_check, n_threads=oracle_threads())
     o.set_kv(K.cpu(), V.cpu())
-    fed = np.concatenate([start, toks_d[:n_check - 1]]).astype(np.int32)
     ref = o.forced(fed, w.kv_len)
-    mx, rel = check_logits(lg[:n_check], ref, name + " follow")
+    g = lg[:n_check]
+    mx_e, rel_e = check_logits(g, ex, name + " vs exact")
+    mx_o, rel_o = check_logits(g, ref, name + " vs oracle", rel_bound_from_exact(ref, ex),
+                               atol_bound_from_exact(ref, ex))
     check_tokens_against_logits(toks_d[:n_check], ref, name + " follow")
-    print("%s: %d steps in follow mode, max|d| %.3g, max rel-L2 %.3g" % (name, n_check, mx, rel))
+    o_ex = rel_l2(ref, ex)
+    print("\n%s | %d follow-mode steps | GPU vs exact: max|d| %.2e, max rel-L2 %.2e | GPU vs oracle: max|d| %.2e, "
+          "max rel-L2 %.2e, steps above 1e-3: %d | oracle vs exact: max rel-L2 %.2e, steps above 1e-3: %d"
+          % (name, n_check, mx_e, rel_e, mx_o, rel_o, int((rel_l2(g, ref) > REL_L2).sum()), o_ex.max(),
+             int((o_ex > REL_L2).sum())))

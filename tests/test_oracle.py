@@ -10,7 +10,7 @@ import pytest
 import torch
 
 import oracle
-from oracle import naive
+from oracle import exact, naive
 import synth
 
 
@@ -221,6 +221,23 @@ def test_decode_with_prefilled_cache_reproduces_causal_forward(tiny, tiny_weight
     got = _forced_run(tiny, tiny_weights, toks, pos0=P, kv=(K, V))
     want = naive.causal_forward(tiny.dims(), tiny_weights, toks, pos0=P, kv_prefix=(K, V))
     assert np.abs(got - want).max() <= 1e-4 * np.abs(want).max()
+
+
+@pytest.mark.parametrize("prefix", [0, 40])
+def test_torch_fp64_forward_matches_numpy_fp64_forward(tiny, tiny_weights, prefix):
+    """oracle.exact (torch, one layer widened at a time, used on a GPU for the large models)
+    states the same float64 forward as naive.causal_forward (numpy): they agree to float64
+    rounding on the tiny model, from position 0 and over a pre-filled cache. A transposed
+    operand, a wrong group index or a dropped term in either moves logits by O(1)."""
+    toks = synth.make_tokens(tiny, 12).numpy()
+    kv = None
+    if prefix:
+        K, V = synth.make_kv(tiny, seed=2, device="cpu", n_pos=prefix)
+        kv = (K, V)
+    want = naive.causal_forward(tiny.dims(), tiny_weights, toks, pos0=prefix, kv_prefix=kv)
+    got = exact.causal_forward(tiny.dims(), tiny_weights, toks, pos0=prefix, kv_prefix=kv)
+    assert got.shape == want.shape
+    assert np.abs(got - want).max() <= 1e-10 * np.abs(want).max()
 
 
 def _llama(dims, weights):
