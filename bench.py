@@ -33,11 +33,11 @@ METRIC = "batch-1 decode tokens/s on 1 B200 (2B bf16) and % of HBM-bandwidth roo
 SPEC_HBM_GBS = 8000.0          # B200 HBM3e specification
 # DRAM bytes per algorithmic byte of the monokernel, from one ncu capture
 # (dram__bytes_read.sum + dram__bytes_write.sum of one launch decoding 8 tokens of the 2B model
-# at a 4k context; profiles/monokernel_2b-4k_8tok_counters.md). It holds for the kernel source
-# it was taken on only: when csrc/kd_kernel.cu no longer has this SHA-256, traffic is null.
-TRAFFIC_CAPTURE = {"kernel_sha256": "1ce29b35780aaf3994a3ec3d2bbc969f2b70c587fbff10571c48e468f432e7d7",
-                   "dram_bytes": 32994343168.0 + 64696064.0, "algorithmic_bytes": 32998424576.0}
-FALLBACK_HBM_GBS = 6650.0       # earlier measurement on this machine, if no measured peaks file
+# at a 4k context, `--workload 2b-4k --n-gen 8`). It holds for the kernel source it was taken on
+# only: when csrc/kd_kernel.cu no longer has this SHA-256, traffic is null.
+TRAFFIC_CAPTURE = {"kernel_sha256": "ea5611cbdbb76ba1c534d5ae5909df76001c23f568d03a152bd072a2f39e12f6",
+                   "dram_bytes": 32998984000.0 + 125110528.0, "algorithmic_bytes": 32998424576.0}
+FALLBACK_HBM_GBS = 6650.0       # an earlier B200 copy measurement, used without a measured peaks file
 
 
 def kernel_source_sha256() -> str:
@@ -82,6 +82,8 @@ def parse():
     ap.add_argument("--impl", default="kernel", choices=["kernel", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-tokens", type=int, default=8)
+    ap.add_argument("--phase-trace", action="store_true",
+                    help="instead of the benchmark line, print where one launch spends its time (per-phase trace)")
     return ap.parse_args()
 
 
@@ -224,6 +226,119 @@ def reference_arm(args, w):
     print(json.dumps(line), flush=True)
 
 
+PHASES = ["qkv", "attention", "o_proj", "gate_up", "down", "lm_head"]
+
+
+def phase_trace(dec, w, d_start, warmup):
+    """Where one launch spends its time, from the kernel's per-phase trace (kd_set_trace):
+    one traced launch of the workload with every CTA recording, next to the median of three
+    untraced ones. Returns a dict (printed as one JSON line); see summarize_trace."""
+    import torch
+    import persistent_monokernel_sm_b200 as kd
+    L, steps = w.dims()["n_layers"], w.n_steps
+    rows = 5 * L * steps + steps + 2
+    grid = dec.info().grid
+    buf = torch.zeros(grid * rows * 8, dtype=torch.int64, device=d_start.device)
+
+    def launch(traced):
+        kd.kd_set_trace(dec.h, buf.data_ptr() if traced else None, buf.numel(), 1)
+        dec.reset(d_start, w.start_pos)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(dec.stream)
+        dec.decode(w.n_gen)
+        e1.record(dec.stream)
+        dec.sync()
+        return e0.elapsed_time(e1)
+
+    for _ in range(max(1, warmup)):
+        launch(False)
+    plain_ms = statistics.median(launch(False) for _ in range(3))
+    traced_ms = launch(True)
+    kd.kd_set_trace(dec.h, None, 0, 1)
+    tr = buf.cpu().numpy().reshape(grid, rows, 8)
+    out = summarize_trace(tr, traced_ms)
+    out.update({"workload": w.name, "tokens": w.n_gen, "grid": grid, "launch_ms": plain_ms,
+                "traced_launch_ms": traced_ms, "launches_per_token": 1.0 / w.n_gen})
+    return {"phase_trace": out}
+
+
+def summarize_trace(tr, traced_ms):
+    """Per-phase times and time fractions of one traced launch.
+
+    tr: [grid][rows][8] int64, the kernel's trace rows (per phase: id = step << 16 | layer << 4
+    | phase, begin, inputs ready, compute done, end, cycles waiting for stages, first and last
+    stage ready), the producer's row last. Inputs ready ends the cross-CTA wait of a phase that
+    follows a sync (Q/K/V after layer 0, gate/up, LM head: the wait for the counter plus the
+    fold of the summed delta into the residual and its norm) or the poll on the kv head's
+    exchange words (attention: the step's q/k/v; output projection: the attention records). A
+    CTA without an attention piece stamps neither mark in that phase (all of it counts as
+    compute). The step boundary (the wait for the previous step's argmax, the embedding
+    gather) lies between a step's last phase and the next step's first and counts as sync
+    wait. Steps >= 1 are averaged; SM cycles become time by the launch's measured duration."""
+    import numpy as np
+    grid, rows = tr.shape[0], tr.shape[1]
+    body = tr[:, :rows - 1, :].astype(np.int64)
+    live = []
+    for c in range(grid):
+        b = body[c][body[c][:, 1] != 0].copy()
+        b[:, 2] = np.where(b[:, 2] == 0, b[:, 1], b[:, 2])
+        b[:, 3] = np.where(b[:, 3] == 0, b[:, 4], b[:, 3])
+        live.append(b)
+    span_cyc = [b[:, 4].max() - b[:, 1].min() for b in live if len(b)]
+    mhz = float(np.median(span_cyc)) / (traced_ms * 1e3)  # SM cycles per microsecond
+    keys = ("wait", "compute", "tail", "stage_wait", "total", "first_stage", "stage_span", "after_last_stage")
+    per = {n: {k: [] for k in keys} for n in PHASES}
+    spans, boundary, other_gaps, sync_wait, xchg_wait, stage_wait, tails = [], [], [], [], [], [], []
+    for b in live:
+        ids = b[:, 0]
+        step, layer, ph = ids >> 16, (ids >> 4) & 0xfff, ids & 15
+        sel = step >= 1
+        if not sel.any():
+            continue
+        bs, phs, lays, sts = b[sel], ph[sel], layer[sel], step[sel]
+        spans.append((bs[:, 4].max() - bs[:, 1].min()) / mhz)
+        for k, n in enumerate(PHASES):
+            x = bs[phs == k]
+            if not len(x):
+                continue
+            d = per[n]
+            d["wait"].append(((x[:, 2] - x[:, 1]) / mhz).mean())
+            d["compute"].append(((x[:, 3] - x[:, 2]) / mhz).mean())
+            d["tail"].append(((x[:, 4] - x[:, 3]) / mhz).mean())
+            d["stage_wait"].append((x[:, 5] / mhz).mean())
+            d["total"].append(((x[:, 4] - x[:, 1]) / mhz).mean())
+            hs = x[x[:, 6] != 0]
+            if len(hs):
+                d["first_stage"].append(((hs[:, 6] - hs[:, 2]) / mhz).mean())
+                d["stage_span"].append(((hs[:, 7] - hs[:, 6]) / mhz).mean())
+                d["after_last_stage"].append(((hs[:, 3] - hs[:, 7]) / mhz).mean())
+        w_in = (bs[:, 2] - bs[:, 1]) / mhz
+        after_sync = ((phs == 0) & (lays > 0)) | (phs == 3) | (phs == 5)
+        gaps = (bs[1:, 1] - bs[:-1, 4]) / mhz
+        new_step = sts[1:] != sts[:-1]
+        nsteps = max(1, len(set(sts.tolist())) - 1)
+        boundary.append(gaps[new_step].sum() / nsteps)
+        other_gaps.append(gaps[~new_step].sum() / nsteps)
+        sync_wait.append(w_in[after_sync].sum() + gaps[new_step].sum())
+        xchg_wait.append(w_in[(phs == 1) | (phs == 2)].sum())
+        stage_wait.append((bs[:, 5] / mhz).sum())
+        tails.append(((bs[:, 4] - bs[:, 3]) / mhz).sum())
+    span = float(np.mean(spans))
+    return {
+        "sm_cycles_per_us": mhz,
+        "us_per_phase": {n: {k: float(np.mean(v)) for k, v in d.items() if v} for n, d in per.items() if d["total"]},
+        "fraction_of_time": {
+            "cross_cta_sync_wait": float(np.mean(sync_wait)) / span,
+            "kv_head_exchange_wait": float(np.mean(xchg_wait)) / span,
+            "stage_wait_in_compute": float(np.mean(stage_wait)) / span,
+            "phase_tails": float(np.mean(tails)) / span,
+        },
+        "step_boundary_us": float(np.mean(boundary)),
+        "between_phases_us_per_step": float(np.mean(other_gaps)),
+        "step_boundary_us_max_over_ctas": float(np.max(boundary)),
+    }
+
+
 def workload_config(w, n_gen):
     return {"workload": w.name, "n_layers": w.n_layers, "d_model": w.d_model, "n_heads": w.n_heads,
             "n_kv_heads": w.n_kv_heads, "head_dim": w.head_dim, "ffn_dim": w.ffn_dim, "vocab": w.vocab,
@@ -275,6 +390,14 @@ def main():
     def step():
         dec.reset(d_start, w.start_pos)
         dec.decode(w.n_gen, out=tok_out)
+
+    if args.phase_trace:
+        if rank == 0:
+            print(json.dumps(phase_trace(dec, w, d_start, args.warmup)), flush=True)
+        dec.close()
+        if world > 1:
+            dist.destroy_process_group()
+        return
 
     for _ in range(args.warmup):
         step()

@@ -6,8 +6,9 @@
 // cudaMalloc after start-up, a host that only hands the library pre-registered buffers, and
 // code paths where an allocation could fail or stall mid-request. Such a caller still owns
 // the weights and the KV cache (the handle's arena from kd_create) and its own input and
-// output buffers; the activation vectors, split-K attention partials, control words and the
-// pending-token list live here instead of in the arena's scratch region.
+// output buffers; the split-K sums, the exchange words (Q/K/V outputs and attention records),
+// the control words and the pending-token list live here instead of in the arena's scratch
+// region.
 #include <cuda_runtime.h>
 #include <mutex>
 #include <stdio.h>
