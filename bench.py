@@ -34,17 +34,21 @@ SPEC_HBM_GBS = 8000.0          # B200 HBM3e specification
 # DRAM bytes per algorithmic byte of the monokernel, from one ncu capture
 # (dram__bytes_read.sum + dram__bytes_write.sum of one launch decoding 8 tokens of the 2B model
 # at a 4k context, `--workload 2b-4k --n-gen 8`). It holds for the kernel source it was taken on
-# only: when csrc/kd_kernel.cu no longer has this SHA-256, traffic is null.
+# only: when csrc/kd_kernel.cu + csrc/kd_layout.h no longer hash to this SHA-256, traffic is
+# null.
 TRAFFIC_CAPTURE = {"kernel_sha256": "ea5611cbdbb76ba1c534d5ae5909df76001c23f568d03a152bd072a2f39e12f6",
                    "dram_bytes": 32998984000.0 + 125110528.0, "algorithmic_bytes": 32998424576.0}
 FALLBACK_HBM_GBS = 6650.0       # an earlier B200 copy measurement, used without a measured peaks file
 
 
 def kernel_source_sha256() -> str:
+    """SHA-256 of the kernel source and its launch-shape header, concatenated."""
     import hashlib
-    path = os.path.join(ROOT, "persistent_monokernel_sm_b200", "csrc", "kd_kernel.cu")
-    with open(path, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()
+    h = hashlib.sha256()
+    for name in ("kd_kernel.cu", "kd_layout.h"):
+        with open(os.path.join(ROOT, "persistent_monokernel_sm_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
 
 
 def launch_traffic(bytes_launch: float):

@@ -543,12 +543,16 @@ __device__ __forceinline__ void gemv_rows(const Params& P, const Smem& sm, const
     const size_t rowbytes = (size_t)d * 2;
     const int nst = (nrows + gr - 1) / gr;
 
+    // Lanes 4..7 of each quarter-warp read the second half of their 8 activations first, so
+    // that each 16-byte load of a quarter-warp touches 8 different bank groups.
     float xr[NCH][8];
+    const int hsw = (lane >> 2) & 1;
 #pragma unroll
     for (int i = 0; i < NCH; ++i) {
         const int k = sl * slen + (lane + 32 * i) * 8;
-        const float4 a = *reinterpret_cast<const float4*>(sm.x + k);
-        const float4 b = *reinterpret_cast<const float4*>(sm.x + k + 4);
+        const float4 f = *reinterpret_cast<const float4*>(sm.x + k + 4 * hsw);
+        const float4 z = *reinterpret_cast<const float4*>(sm.x + k + 4 - 4 * hsw);
+        const float4 a = hsw ? z : f, b = hsw ? f : z;
         const uint4 g = lds128(sm.gain + k);
         xr[i][0] = (a.x * scale) * bf_lo(g.x), xr[i][1] = (a.y * scale) * bf_hi(g.x);
         xr[i][2] = (a.z * scale) * bf_lo(g.y), xr[i][3] = (a.w * scale) * bf_hi(g.y);
