@@ -36,8 +36,8 @@ SPEC_HBM_GBS = 8000.0          # B200 HBM3e specification
 # at a 4k context, `--workload 2b-4k --n-gen 8`). It holds for the kernel source it was taken on
 # only: when csrc/kd_kernel.cu + csrc/kd_layout.h no longer hash to this SHA-256, traffic is
 # null.
-TRAFFIC_CAPTURE = {"kernel_sha256": "ea5611cbdbb76ba1c534d5ae5909df76001c23f568d03a152bd072a2f39e12f6",
-                   "dram_bytes": 32998984000.0 + 125110528.0, "algorithmic_bytes": 32998424576.0}
+TRAFFIC_CAPTURE = {"kernel_sha256": "ec508df3ae4685a0249ddbe2b2292417377b44b78bdaf92c1c8d238a2682996f",
+                   "dram_bytes": 32999400000.0 + 126809856.0, "algorithmic_bytes": 32998424576.0}
 FALLBACK_HBM_GBS = 6650.0       # an earlier B200 copy measurement, used without a measured peaks file
 
 
