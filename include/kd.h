@@ -154,6 +154,19 @@ int kd_generate(kd_ctx *ctx, const int32_t *h_tokens, int32_t n_tokens, int32_t 
  * KD_ETIMEOUT and the handle needs kd_reset. Returns KD_EINVAL for ns < 1. */
 int kd_set_timeout(kd_ctx *ctx, int64_t ns);
 
+/* Token choice of later kd_decode / kd_generate / kd_decode_noalloc calls. temperature 0
+ * (the default) picks the greedy argmax. temperature > 0 draws each generated token from
+ * softmax(logits / temperature) inside the kernel ("3000 tokens per second", aikraft.ru,
+ * section 04 "Monokernel": sampling stays on the GPU): the argmax over the vocabulary of
+ * logit_i * (1/temperature) + g_i, g_i = -log(-log(u_i)) (the Gumbel-max rule, an exact draw),
+ * in fp32, lowest index on a tie. u_i comes from the counter-based generator Philox4x32-10
+ * (Salmon et al., SC 2011) with key (seed mod 2^32, seed div 2^32) and counter
+ * (i div 4, position, 0, 0), output word i mod 4, u = (top 24 bits + 0.5) / 2^24; the position is
+ * the absolute KV position of the step, so a request draws the same tokens however it is split
+ * into calls. Logits written to d_logits_out stay the raw logits. Returns KD_EINVAL for a
+ * negative or non-finite temperature. */
+int kd_set_sampling(kd_ctx *ctx, float temperature, uint64_t seed);
+
 /* Wait for the stream, then return the device status of the last decode (KD_OK,
  * KD_ETIMEOUT, KD_ETOKEN) or a CUDA error. */
 int kd_sync(kd_ctx *ctx);

@@ -14,7 +14,7 @@ import os
 
 __all__ = ["KdError", "kd_config", "kd_weights", "kd_info", "load_library", "Decoder", "config_from",
            "kd_arena_bytes", "kd_step_bytes", "kd_create", "kd_load_weights", "kd_set_kv", "kd_reset",
-           "kd_decode", "kd_generate", "kd_sync", "kd_position", "kd_set_trace", "kd_set_timeout", "kd_decode_noalloc", "kd_get_info", "kd_kv_ptr",
+           "kd_decode", "kd_generate", "kd_sync", "kd_position", "kd_set_trace", "kd_set_timeout", "kd_set_sampling", "kd_decode_noalloc", "kd_get_info", "kd_kv_ptr",
            "kd_last_error", "kd_strerror", "kd_destroy", "LIB_PATH", "ERRORS"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkd.so")
@@ -77,6 +77,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "kd_position": (ctypes.c_int32, [_P]),
         "kd_set_trace": (ctypes.c_int, [_P, _P, ctypes.c_int64, ctypes.c_int32]),
         "kd_set_timeout": (ctypes.c_int, [_P, ctypes.c_int64]),
+        "kd_set_sampling": (ctypes.c_int, [_P, ctypes.c_float, ctypes.c_uint64]),
         "kd_decode_noalloc": (ctypes.c_int, [_P, _P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, _P, _P]),
         "kd_get_info": (ctypes.c_int, [_P, ctypes.POINTER(kd_info)]),
         "kd_kv_ptr": (_P, [_P, ctypes.c_int32, ctypes.c_int32]),
@@ -151,6 +152,11 @@ def kd_decode_noalloc(h, d_tokens: int, n_tokens: int, kv_len: int, n_gen: int, 
 
 def kd_set_timeout(h, ns: int) -> int:
     return _check(h, load_library().kd_set_timeout(h, ns), "kd_set_timeout")
+
+
+def kd_set_sampling(h, temperature: float, seed: int) -> int:
+    return _check(h, load_library().kd_set_sampling(h, float(temperature), int(seed) & 0xFFFFFFFFFFFFFFFF),
+                  "kd_set_sampling")
 
 
 def kd_set_trace(h, d_buf: int | None, n_words: int, every: int) -> int:
@@ -269,6 +275,10 @@ class Decoder:
 
     def sync(self):
         kd_sync(self.h)
+
+    def set_sampling(self, temperature: float, seed: int = 0):
+        """Greedy at temperature 0 (the default); else in-kernel draws from softmax(logits / T)."""
+        kd_set_sampling(self.h, temperature, seed)
 
     def position(self) -> int:
         return kd_position(self.h)

@@ -99,6 +99,8 @@ struct kd_ctx {
     int pos, n_pending;
     long long launches;
     long long timeout_ns;
+    float inv_temp;            // 0: greedy
+    unsigned long long seed;   // sampling stream
     uint32_t tag;  // tag base of the next launch (advanced by the tagged phases each launch runs)
     unsigned long long* trace;
     int trace_every, trace_rows;
@@ -217,6 +219,8 @@ int kd_internal_view(kd_ctx* c, kd_ctx_view* v) {
     v->pieces = c->pieces, v->blk = c->blk, v->work_floats = c->work_floats, v->hin_floats = c->hin_floats;
     v->timeout_ns = c->timeout_ns;
     v->has_weights = c->has_weights;
+    v->inv_temp = c->inv_temp;
+    v->seed = c->seed;
     return KD_OK;
 }
 
@@ -236,6 +240,9 @@ void fill_launch_shape(const kd_ctx_view& v, Params& p) {
     p.work_floats = v.work_floats;
     p.hin_floats = v.hin_floats;
     p.timeout_ns = v.timeout_ns;
+    p.inv_temp = v.inv_temp;
+    p.seed_lo = (uint32_t)(v.seed & 0xffffffffull);
+    p.seed_hi = (uint32_t)(v.seed >> 32);
 }
 }  // namespace kd
 
@@ -519,6 +526,15 @@ int kd_set_trace(kd_ctx* c, unsigned long long* d_buf, int64_t n_words, int32_t 
     c->trace = d_buf;
     c->trace_every = every;
     c->trace_rows = (int)rows;
+    return KD_OK;
+}
+
+int kd_set_sampling(kd_ctx* c, float temperature, uint64_t seed) {
+    if (!c) return KD_EINVAL;
+    if (!(temperature >= 0.0f) || !isfinite(temperature))
+        return fail(c, KD_EINVAL, "kd_set_sampling: temperature must be finite and >= 0");
+    c->inv_temp = temperature > 0.0f ? 1.0f / temperature : 0.0f;
+    c->seed = seed;
     return KD_OK;
 }
 

@@ -1045,7 +1045,7 @@ __device__ __forceinline__ void run_attention(const Params& P, const Smem& sm, c
 }
 
 // Output-projection inputs: combine the attention records of every piece of this CTA's kv
-// head for its own output dims (pieces in order: max-rescaled sums) into sm.hin. Returns the
+// head for its own output dims (max-rescaled sums over the pieces) into sm.hin. Returns the
 // number of dims (rows of the transposed output projection this CTA multiplies).
 template <int HD>
 __device__ __forceinline__ int oproj_inputs(const Params& P, const Smem& sm, const unsigned long long* ctl, int t, int l,
@@ -1081,17 +1081,27 @@ __device__ __forceinline__ int oproj_inputs(const Params& P, const Smem& sm, con
     }
     ok = consumer_sync_and(ok);
     tr.mark(2);
-    for (int j = threadIdx.x; j < ncol; j += kConsumerThreads) {
+    // one warp per output dim, its lanes over the pieces; the max and the two sums are
+    // reduced across the warp (a fixed shuffle tree)
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int j = warp; j < ncol; j += kConsumerWarps) {
         const int col = c0 + j, hi = col / HD - h0;
         float M = -INFINITY;
-        for (int pi = 0; pi < A; ++pi) M = fmaxf(M, stage[pi * W + 2 * hi]);
+        for (int pi = lane; pi < A; pi += 32) M = fmaxf(M, stage[pi * W + 2 * hi]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
         float L = 0.f, o = 0.f;
-        for (int pi = 0; pi < A; ++pi) {
+        for (int pi = lane; pi < A; pi += 32) {
             const float f = exp2f(stage[pi * W + 2 * hi] - M);  // 0 for an empty piece
             L = fmaf(stage[pi * W + 2 * hi + 1], f, L);
             o = fmaf(stage[pi * W + 2 * nh + j], f, o);
         }
-        sm.hin[j] = o / L;
+#pragma unroll
+        for (int s2 = 16; s2 > 0; s2 >>= 1) {
+            L += __shfl_xor_sync(0xffffffffu, L, s2);
+            o += __shfl_xor_sync(0xffffffffu, o, s2);
+        }
+        if (lane == 0) sm.hin[j] = o / L;
     }
     consumer_sync();
     return ncol;
@@ -1280,6 +1290,31 @@ struct Producer {
 
 // ------------------------------------------------------------------ the kernel
 
+// ---- temperature sampling: the Gumbel-max draw from softmax(logits / T)
+//
+// Philox4x32-10 (Salmon, Moraes, Dror and Shaw, "Parallel random numbers: as easy as 1, 2, 3",
+// SC 2011): a 128-bit counter, a 64-bit key, ten rounds of two 32x32 -> 64-bit products, the
+// key bumped between rounds by the two Weyl constants.
+__device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1) {
+#pragma unroll
+    for (int r = 0; r < 10; ++r) {
+        if (r > 0) k0 += 0x9E3779B9u, k1 += 0xBB67AE85u;
+        const uint32_t hi0 = __umulhi(0xD2511F53u, c.x), lo0 = 0xD2511F53u * c.x;
+        const uint32_t hi1 = __umulhi(0xCD9E8D57u, c.z), lo1 = 0xCD9E8D57u * c.z;
+        c = make_uint4(hi1 ^ c.y ^ k0, lo1, hi0 ^ c.w ^ k1, lo0);
+    }
+    return c;
+}
+// logit * (1/T) + g for vocabulary index i at absolute position pos, g = -log(-log(u)) with u
+// the (i mod 4)-th word of Philox((i div 4, pos, 0, 0), seed): its top 24 bits + 0.5, / 2^24.
+__device__ __forceinline__ float gumbel_perturbed(const Params& P, float y, int i, int pos) {
+    const uint4 w = philox4x32_10(make_uint4((uint32_t)i >> 2, (uint32_t)pos, 0u, 0u), P.seed_lo, P.seed_hi);
+    const int q = i & 3;
+    const uint32_t x = q == 0 ? w.x : q == 1 ? w.y : q == 2 ? w.z : w.w;
+    const float u = ((float)(x >> 8) + 0.5f) * 5.9604644775390625e-8f;  // 2^-24
+    return y * P.inv_temp - logf(-logf(u));
+}
+
 __device__ __forceinline__ unsigned long long argmax_key(float v, int idx) {
     uint32_t u = __float_as_uint(v);
     u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
@@ -1423,7 +1458,8 @@ __global__ void __launch_bounds__(kThreads, 1) monokernel(const __grid_constant_
                     for (int i = tid; i < g.v1 - g.v0; i += kConsumerThreads) {
                         const float y = row_value(sm, P.sh.gs, i);
                         if (P.dump) __stcg(P.logits_out + (size_t)t * dm.V + g.v0 + i, y);
-                        const unsigned long long key = argmax_key(y, g.v0 + i);
+                        const float z = P.inv_temp > 0.f ? gumbel_perturbed(P, y, g.v0 + i, p) : y;
+                        const unsigned long long key = argmax_key(z, g.v0 + i);
                         best = key > best ? key : best;
                     }
 #pragma unroll

@@ -127,6 +127,9 @@ struct Params {
     int dump;       // write logits of every step
     int32_t* tokens_out;
     float* logits_out;
+    // token choice: greedy when inv_temp == 0, else the Gumbel-max draw with this seed
+    float inv_temp;
+    uint32_t seed_lo, seed_hi;
     // launch shape
     int nb;         // CTAs
     int ns;         // pipeline stages
@@ -160,6 +163,8 @@ struct kd_ctx_view {
     int device, nb, smem, ns, pieces, blk, work_floats, hin_floats;
     long long timeout_ns;
     bool has_weights;
+    float inv_temp;
+    unsigned long long seed;
 };
 int monokernel_smem_bytes(const Params& p);
 int monokernel_occupancy(const Dims& dm, int smem_bytes, int* blocks_per_sm);

@@ -83,6 +83,7 @@ def test_calls_on_a_null_handle_are_refused(kd):
     assert lib.kd_decode_noalloc(None, None, 1, 0, 1, None, None) == -1
     assert kd.kd_strerror(-6).startswith("device-side wait")
     assert lib.kd_set_timeout(None, 1000) == -1
+    assert lib.kd_set_sampling(None, 0.5, 1) == -1
 
 
 def test_step_bytes_equal_the_bytes_the_oracle_reads(kd, tiny, tiny_weights):
