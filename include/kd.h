@@ -95,9 +95,12 @@ typedef struct kd_info {
     int64_t weight_bytes;  /* bytes of the weights inside the arena */
     int64_t kv_bytes;      /* bytes of the KV cache inside the arena */
     int64_t launches;      /* kernel launches made through this handle so far */
-    int64_t ctl_offset;    /* byte offset of the control words in the arena (word 0: the
-                              monotonic 64-bit count of cross-CTA sync arrivals); exposed for
+    int64_t ctl_offset;    /* byte offset of the control words in the arena; exposed for
                               diagnostics and tests, not to be written while a decode runs */
+    int32_t sync_replicas; /* copies of the monotonic 64-bit count of cross-CTA sync arrivals:
+                              2 when kd_create found the two dies of a B200 (every CTA adds to
+                              both, polls the one on its own die), else 1 */
+    int64_t sync_offset[2]; /* byte offsets of those copies in the arena (equal when 1) */
 } kd_info;
 
 typedef struct kd_ctx kd_ctx;

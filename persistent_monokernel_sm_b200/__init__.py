@@ -41,7 +41,8 @@ class kd_weights(ctypes.Structure):
 class kd_info(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in ("grid", "threads", "smem_bytes", "stages", "stage_bytes",
                                                "attn_pieces")] + \
-               [(n, ctypes.c_int64) for n in ("arena_bytes", "weight_bytes", "kv_bytes", "launches", "ctl_offset")]
+               [(n, ctypes.c_int64) for n in ("arena_bytes", "weight_bytes", "kv_bytes", "launches", "ctl_offset")] + \
+               [("sync_replicas", ctypes.c_int32), ("sync_offset", ctypes.c_int64 * 2)]
 
 
 class KdError(RuntimeError):

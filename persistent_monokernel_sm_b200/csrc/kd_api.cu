@@ -1,6 +1,7 @@
 // kd_api.cu -- host side of libkd: configuration checks, the arena layout, weight repacking
 // into the streaming layout, and the C ABI declared in include/kd.h.
 #include <cuda_runtime.h>
+#include <algorithm>
 #include <vector>
 #include <math.h>
 #include <stdarg.h>
@@ -78,10 +79,39 @@ Layout make_layout(const Dims& d) {
     y.qkv = take((size_t)d.qkv_rows * 8);                          // tagged q / k / v of the step
     y.rec = take((size_t)kMaxGrid * d.r * (d.hd + 2) * 8);         // tagged attention records
     y.ctl = take((size_t)kCtlWords * 8);
+    y.syncw = take(sync_region_bytes());
+    y.dietab = take(kMaxSmid);
     y.tokens_in = take((size_t)d.S * 4);
     y.tokens_out = take((size_t)d.S * 4);  // staging for kd_generate
     y.total = off;
     return y;
+}
+
+// End of the scratch that starts at zero and is cleared after a failed run: the split-K
+// buffers, the tagged words, the control words and the sync counter replicas.
+size_t scratch_end(const Layout& y) { return y.syncw + sync_region_bytes(); }
+
+// Die probe, run once by kd_create: each CTA records its SM id and, for each of the ncand
+// candidate counter words (kDieBlock bytes apart), the shortest round trip of a few atomics
+// that add 0. Its outputs go to a scratch region of the arena that is cleared afterwards.
+__global__ void die_probe(unsigned long long* cand, int ncand, int* smid_out, unsigned int* lat_out) {
+    if (threadIdx.x != 0) return;
+    uint32_t sm;
+    asm volatile("mov.u32 %0, %%smid;" : "=r"(sm));
+    smid_out[blockIdx.x] = (int)sm;
+    for (int j = 0; j < ncand; ++j) {
+        unsigned long long* w = cand + (size_t)j * (kDieBlock / 8);
+        long long best = 1LL << 62;
+        for (int r = 0; r < 6; ++r) {
+            const long long t0 = clock64();
+            unsigned long long old, dep;
+            asm volatile("atom.relaxed.gpu.global.add.u64 %0, [%1], 0;" : "=l"(old) : "l"(w) : "memory");
+            asm volatile("shr.b64 %0, %1, 63;" : "=l"(dep) : "l"(old));  // the clock waits for the answer
+            const long long dt = clock64() + (long long)dep - t0;
+            if (r > 0 && dt < best) best = dt;
+        }
+        lat_out[blockIdx.x * ncand + j] = (unsigned int)(best > 0xffffffffLL ? 0xffffffffu : best);
+    }
 }
 
 }  // namespace
@@ -101,6 +131,8 @@ struct kd_ctx {
     long long timeout_ns;
     float inv_temp;            // 0: greedy
     unsigned long long seed;   // sampling stream
+    size_t sync_off[2];        // sync counter replicas (arena byte offsets)
+    int nsync;
     uint32_t tag;  // tag base of the next launch (advanced by the tagged phases each launch runs)
     unsigned long long* trace;
     int trace_every, trace_rows;
@@ -221,6 +253,8 @@ int kd_internal_view(kd_ctx* c, kd_ctx_view* v) {
     v->has_weights = c->has_weights;
     v->inv_temp = c->inv_temp;
     v->seed = c->seed;
+    v->sync_off[0] = c->sync_off[0], v->sync_off[1] = c->sync_off[1];
+    v->nsync = c->nsync;
     return KD_OK;
 }
 
@@ -243,6 +277,8 @@ void fill_launch_shape(const kd_ctx_view& v, Params& p) {
     p.inv_temp = v.inv_temp;
     p.seed_lo = (uint32_t)(v.seed & 0xffffffffull);
     p.seed_hi = (uint32_t)(v.seed >> 32);
+    p.sync_off[0] = v.sync_off[0], p.sync_off[1] = v.sync_off[1];
+    p.nsync = v.nsync;
 }
 }  // namespace kd
 
@@ -265,6 +301,55 @@ double kd_step_bytes(const kd_config* cfg, int64_t kv_positions, int with_head) 
     if (with_head) elems += d + V * d;
     const double kv = L * Hkv * (double)kv_positions * hd * 2;  // K and V rows
     return 2.0 * (elems + kv);
+}
+
+// Which die owns which counter word, and which replica is local to each SM. The candidates
+// are kDieBlock-aligned words of the sync region; candidate 0 is replica 0; replica 1 is the
+// first candidate whose round trips differ from candidate 0's by more than 1.4x for the
+// median CTA (the two are then homed on different dies); each SM takes the replica with the
+// shorter round trip. With no such candidate (one die, or a probe that saw no difference)
+// there is one replica. Correctness never depends on the outcome: every CTA adds to every
+// replica, and a wrong local choice only costs latency.
+static int probe_dies(kd_ctx* c) {
+    const uintptr_t a0 = (uintptr_t)(c->arena + c->lay.syncw);
+    const uintptr_t al = (a0 + kDieBlock - 1) & ~(uintptr_t)(kDieBlock - 1);
+    const size_t base = (size_t)(al - (uintptr_t)c->arena);
+    c->sync_off[0] = c->sync_off[1] = base;
+    c->nsync = 1;
+    const int nb = c->nb, K = kDieCandidates;
+    // outputs in the attention-record scratch (cleared below, before any decode)
+    int* d_smid = reinterpret_cast<int*>(c->arena + c->lay.rec);
+    unsigned int* d_lat = reinterpret_cast<unsigned int*>(c->arena + c->lay.rec + 4096);
+    if ((size_t)4096 + (size_t)nb * K * 4 > (size_t)kMaxGrid * c->dm.r * (c->dm.hd + 2) * 8)
+        return fail(c, KD_EINVAL, "die probe: scratch too small");
+    die_probe<<<nb, 32, 0, c->stream>>>(reinterpret_cast<unsigned long long*>(c->arena + base), K, d_smid, d_lat);
+    std::vector<int> smid(nb);
+    std::vector<unsigned int> lat((size_t)nb * K);
+    KD_CUDA(c, cudaGetLastError());
+    KD_CUDA(c, cudaMemcpyAsync(smid.data(), d_smid, (size_t)nb * 4, cudaMemcpyDeviceToHost, c->stream));
+    KD_CUDA(c, cudaMemcpyAsync(lat.data(), d_lat, (size_t)nb * K * 4, cudaMemcpyDeviceToHost, c->stream));
+    KD_CUDA(c, cudaStreamSynchronize(c->stream));
+    int r1 = -1;
+    for (int j = 1; j < K && r1 < 0; ++j) {
+        std::vector<double> ratio(nb);
+        for (int b = 0; b < nb; ++b) {
+            const double x = lat[(size_t)b * K], y = lat[(size_t)b * K + j];
+            ratio[b] = (x > y ? x : y) / ((x < y ? x : y) > 1.0 ? (x < y ? x : y) : 1.0);
+        }
+        std::nth_element(ratio.begin(), ratio.begin() + nb / 2, ratio.end());
+        if (ratio[nb / 2] > 1.4) r1 = j;
+    }
+    std::vector<uint8_t> tab(kMaxSmid, 0);
+    if (r1 > 0) {
+        for (int b = 0; b < nb; ++b)
+            if (smid[b] >= 0 && smid[b] < kMaxSmid) tab[smid[b]] = lat[(size_t)b * K + r1] < lat[(size_t)b * K] ? 1 : 0;
+        c->sync_off[1] = base + (size_t)r1 * kDieBlock;
+        c->nsync = 2;
+    }
+    KD_CUDA(c, cudaMemcpyAsync(c->arena + c->lay.dietab, tab.data(), kMaxSmid, cudaMemcpyHostToDevice, c->stream));
+    KD_CUDA(c, cudaMemsetAsync(c->arena + c->lay.delta, 0, scratch_end(c->lay) - c->lay.delta, c->stream));
+    KD_CUDA(c, cudaStreamSynchronize(c->stream));
+    return KD_OK;
 }
 
 int kd_create(const kd_config* cfg, void* d_arena, size_t arena_bytes, void* stream, kd_ctx** out) {
@@ -335,10 +420,11 @@ int kd_create(const kd_config* cfg, void* d_arena, size_t arena_bytes, void* str
     if (rc == KD_OK) {
         // Control words, the split-K buffers and the tagged words start at zero: tag 0 is
         // never expected (the first launch's phases carry tags 1, 2, ...).
-        cudaError_t e = cudaMemsetAsync(c->arena + c->lay.delta, 0, c->lay.ctl + (size_t)kCtlWords * 8 - c->lay.delta,
+        cudaError_t e = cudaMemsetAsync(c->arena + c->lay.delta, 0, scratch_end(c->lay) - c->lay.delta,
                                         c->stream);
         if (e != cudaSuccess) rc = fail(c, KD_ECUDA, "cudaMemsetAsync: %s", cudaGetErrorString(e));
     }
+    if (rc == KD_OK) rc = probe_dies(c);
     if (rc != KD_OK) {
         fprintf(stderr, "kd_create: %s\n", c->err);
         free(c);
@@ -426,7 +512,7 @@ static int reset_common(kd_ctx* c, int32_t n_tokens, int32_t kv_len) {
     // (the kernel re-bases its sync count, clears its argmax slots and zeroes the buffers), so
     // they are cleared only after a failed run: the decode path then involves no memset.
     if (c->failed)
-        KD_CUDA(c, cudaMemsetAsync(c->arena + c->lay.delta, 0, c->lay.ctl + (size_t)kCtlWords * 8 - c->lay.delta,
+        KD_CUDA(c, cudaMemsetAsync(c->arena + c->lay.delta, 0, scratch_end(c->lay) - c->lay.delta,
                                    c->stream));
     c->pos = kv_len;
     c->n_pending = n_tokens;
@@ -559,6 +645,9 @@ int kd_get_info(const kd_ctx* c, kd_info* info) {
     info->kv_bytes = (int64_t)c->lay.kv_bytes;
     info->launches = c->launches;
     info->ctl_offset = (int64_t)c->lay.ctl;
+    info->sync_replicas = c->nsync;
+    info->sync_offset[0] = (int64_t)c->sync_off[0];
+    info->sync_offset[1] = (int64_t)c->sync_off[1];
     return KD_OK;
 }
 

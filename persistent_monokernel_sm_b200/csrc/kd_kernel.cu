@@ -449,17 +449,30 @@ __device__ __forceinline__ bool get_word(const unsigned long long* p, uint32_t t
 
 // Arrive at cross-CTA sync k: every consumer thread's atomics of this phase are done (the
 // CTA barrier), then one release add publishes them with the arrival.
-__device__ __forceinline__ void sync_arrive(unsigned long long* ctl) {
+// Arrive at the next cross-CTA sync: after a CTA barrier, thread 0 adds 1 to every replica of
+// the counter with release semantics (one fence, then the adds).
+__device__ __forceinline__ void sync_arrive(const Smem& sm) {
     consumer_sync();
-    if (threadIdx.x == 0) red_release_add_u64(ctl + kCtlSync, 1ull);
+    if (threadIdx.x == 0) {
+        unsigned long long* local = reinterpret_cast<unsigned long long*>(sm.u64[1]);
+        unsigned long long* other = reinterpret_cast<unsigned long long*>(sm.u64[2]);
+        if (other) {
+            asm volatile("fence.acq_rel.gpu;" ::: "memory");
+            asm volatile("red.relaxed.gpu.global.add.u64 [%0], 1;" ::"l"(local) : "memory");
+            asm volatile("red.relaxed.gpu.global.add.u64 [%0], 1;" ::"l"(other) : "memory");
+        } else {
+            red_release_add_u64(local, 1ull);
+        }
+    }
 }
 // Wait until every CTA has arrived at this launch's sync number k (thread 0 polls with
 // acquire loads, the CTA barrier then orders every consumer thread after it). Returns
 // false in every consumer thread when the wait gave up or another wait failed.
-__device__ __noinline__ int sync_spin(const unsigned long long* ctl, uint64_t target, long long timeout_ns, long long k) {
+__device__ __noinline__ int sync_spin(const unsigned long long* ctl, const unsigned long long* counter, uint64_t target,
+                                     long long timeout_ns, long long k) {
     Deadline dl;
     for (uint32_t it = 0;; ++it) {
-        if (ld_acquire_u64(ctl + kCtlSync) >= target) return 1;
+        if (ld_acquire_u64(counter) >= target) return 1;
         if ((it & 31) == 31 && !dl.alive(ctl, timeout_ns, where_code(kWhereSync, (int)(k & 0xff)))) return 0;
     }
 }
@@ -467,7 +480,7 @@ __device__ __forceinline__ bool sync_wait(const Smem& sm, const Params& P, const
                                           bool ok) {
     if (threadIdx.x == 0) {
         const uint64_t target = sm.u64[0] + (uint64_t)(k + 1) * (uint64_t)P.nb;
-        sm.flag[0] = ok ? sync_spin(ctl, target, P.timeout_ns, k) : 0;
+        sm.flag[0] = ok ? sync_spin(ctl, reinterpret_cast<const unsigned long long*>(sm.u64[1]), target, P.timeout_ns, k) : 0;
     }
     consumer_sync();
     return sm.flag[0] != 0;
@@ -1226,7 +1239,8 @@ struct Producer {
         const long long c0 = clock64();
         Deadline dl;
         for (uint32_t it = 0;; ++it) {
-            seen = (long long)((ld_acquire_u64(ctl + kCtlSync) - base) / (uint64_t)P.nb);
+            seen = (long long)((ld_acquire_u64(reinterpret_cast<const unsigned long long*>(sm.u64[1])) - base) /
+                               (uint64_t)P.nb);
             if (seen >= need) break;
             if ((it & 31) == 31 && !dl.alive(ctl, P.timeout_ns, where_code(kWhereKv, 0))) return false;
         }
@@ -1341,10 +1355,18 @@ __global__ void __launch_bounds__(kThreads, 1) monokernel(const __grid_constant_
         }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         cta_geo(P, blockIdx.x, *sm.geo);
+        // The counter replica local to this SM (kd_create measured which die owns which), and
+        // the other one if there are two.
+        uint32_t smid;
+        asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+        const int rep = P.nsync == 2 && smid < (uint32_t)kMaxSmid ? (P.arena[P.lay.dietab + smid] & 1) : 0;
+        uint8_t* ab = const_cast<uint8_t*>(P.arena);
+        sm.u64[1] = reinterpret_cast<unsigned long long>(ab + P.sync_off[rep]);
+        sm.u64[2] = P.nsync == 2 ? reinterpret_cast<unsigned long long>(ab + P.sync_off[rep ^ 1]) : 0ull;
         // Sync count at launch: a multiple of nb (every launch that completed arrived nb times
-        // at each of its syncs) plus arrivals of CTAs already at this launch's first sync
-        // (which cannot complete before this CTA arrives).
-        const uint64_t raw = ld_acquire_u64(ctl + kCtlSync);
+        // at each of its syncs, on every replica) plus arrivals of CTAs already at this launch's
+        // first sync (which cannot complete before this CTA arrives).
+        const uint64_t raw = ld_acquire_u64(reinterpret_cast<const unsigned long long*>(sm.u64[1]));
         sm.u64[0] = raw - raw % (uint64_t)P.nb;
         sm.flag[0] = read_status(ctl);
     }
@@ -1478,7 +1500,7 @@ __global__ void __launch_bounds__(kThreads, 1) monokernel(const __grid_constant_
                         red_max_u64(ctl + kCtlArgmax + 16 * (t % 3), b);
                     }
                     tr.mark(3);
-                    if (ok) sync_arrive(ctl);  // -> sync k: the step's argmax is complete
+                    if (ok) sync_arrive(sm);  // -> sync k: the step's argmax is complete
                     ++k;
                 }
             } else if (ph == kATT) {
@@ -1493,7 +1515,7 @@ __global__ void __launch_bounds__(kThreads, 1) monokernel(const __grid_constant_
                 run_splitk(P, sm, ctl, nrows, sm.hin, delta + (size_t)(k % 3) * dm.d, rg, ok, tr);
                 tr.mark(3);
                 ok = consumer_sync_and(ok);
-                if (ok) sync_arrive(ctl);
+                if (ok) sync_arrive(sm);
                 ++k;
             }
             tr.end();

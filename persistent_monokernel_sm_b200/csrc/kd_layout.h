@@ -26,11 +26,20 @@ constexpr int kMaxModel = 8192;     // d_model
 constexpr int kSmemLimit = 232448;  // opt-in dynamic shared memory per CTA on B200
 
 // Control words (uint64), each on its own 128-byte line.
-constexpr int kCtlSync = 0;     // arrivals at the cross-CTA sums and the argmax, monotonic
+constexpr int kCtlSync = 0;     // the sync counter of kd_decode_noalloc (kd_decode uses Params.sync_off)
 constexpr int kCtlStatus = 16;  // 0 = ok, else an error code (device side)
 constexpr int kCtlWhere = 17;   // where a wait gave up (diagnosis)
 constexpr int kCtlArgmax = 32;  // 3 rotating argmax slots at kCtlArgmax + 16*i
 constexpr int kCtlWords = 80;
+
+// Die-local sync counters. A B200 spreads its SMs and its L2 over two dies; an atomic on a
+// line homed on the far die takes about twice the round trip of one on the near die. kd_create
+// probes kDieCandidates words kDieBlock bytes apart (the die owning a line changes at that
+// granularity or coarser), keeps the first candidate and the first one homed on the other die
+// as the two replicas of the sync counter, and records per SM id which replica is local.
+constexpr int kDieCandidates = 16;
+constexpr int kDieBlock = 2048;
+constexpr int kMaxSmid = 256;
 
 constexpr int kStatusTimeout = 1;  // a device-side wait exceeded its limit
 constexpr int kStatusToken = 2;    // a token id outside [0, vocab) reached the kernel
@@ -60,7 +69,10 @@ struct Layout {
     //   qkv [Hkv][(r + 2) * hd] tagged words -- RoPE'd q, RoPE'd bf16 k, bf16 v of the step
     //   rec [grid][r][hd + 2] tagged words   -- attention piece records (max, sum, acc[hd])
     size_t delta, qkv, rec;
-    size_t ctl, tokens_in, tokens_out;
+    size_t ctl;
+    size_t syncw;   // the die probe candidates / sync counter replicas (kDieBlock-aligned inside)
+    size_t dietab;  // [kMaxSmid] uint8: the replica local to each SM id (written at kd_create)
+    size_t tokens_in, tokens_out;
     size_t weights_end, kv_bytes, total;
 };
 
@@ -101,6 +113,9 @@ inline bool make_shape(int d, Shape* s) {
     return true;
 }
 
+// Bytes reserved for the sync counter replicas (alignment slack included).
+KD_HD inline size_t sync_region_bytes() { return (size_t)(kDieCandidates + 1) * kDieBlock; }
+
 // Cross-CTA sums ("syncs") per decode step: the output projection and the down projection of
 // every layer, then the argmax of the steps that run the LM head (all steps when logits are
 // dumped). Sync k adds into delta buffer k % 3.
@@ -130,6 +145,10 @@ struct Params {
     // token choice: greedy when inv_temp == 0, else the Gumbel-max draw with this seed
     float inv_temp;
     uint32_t seed_lo, seed_hi;
+    // sync counter: nsync replicas (1 or 2) at these arena byte offsets; every CTA adds to all
+    // of them and polls the one local to its SM (lay.dietab)
+    size_t sync_off[2];
+    int nsync;
     // launch shape
     int nb;         // CTAs
     int ns;         // pipeline stages
@@ -165,6 +184,8 @@ struct kd_ctx_view {
     bool has_weights;
     float inv_temp;
     unsigned long long seed;
+    size_t sync_off[2];
+    int nsync;
 };
 int monokernel_smem_bytes(const Params& p);
 int monokernel_occupancy(const Dims& dm, int smem_bytes, int* blocks_per_sm);

@@ -114,6 +114,10 @@ extern "C" int kd_decode_noalloc(kd_ctx* ctx, const int32_t* d_tokens, int32_t n
     p.lay = *v.lay;
     p.lay.delta = rel(o_delta), p.lay.qkv = rel(o_qkv), p.lay.rec = rel(o_rec);
     p.lay.ctl = rel(o_ctl), p.lay.tokens_in = rel(o_tok);
+    // one sync counter, in this call's control words (the handle's die-local replicas stay
+    // the handle's)
+    p.sync_off[0] = p.sync_off[1] = rel(o_ctl) + (size_t)kCtlSync * 8;
+    p.nsync = 1;
     p.steps = steps;
     p.n_pending = n_tokens;
     p.pos0 = kv_len;

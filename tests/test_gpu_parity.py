@@ -226,18 +226,26 @@ def test_wait_limit_reports_timeout_and_recovers(kd):
     assert compare_gpu_runs(ref, again.cpu().numpy(), chosen, "after a timeout") == 16
 
 
+def _sync_offsets(dec):
+    info = dec.info()
+    base = dec._arena_ptr - dec.arena.data_ptr()
+    return sorted({base + info.sync_offset[i] for i in range(info.sync_replicas)})
+
+
 def _write_sync_counter(dec, value):
-    """Set the monotonic sync-arrival counter (control word 0) of an idle handle."""
-    off = dec._arena_ptr - dec.arena.data_ptr() + dec.info().ctl_offset
+    """Set every copy of the monotonic sync-arrival counter of an idle handle."""
     dec.stream.synchronize()
-    dec.arena[off:off + 8].copy_(torch.tensor([value], dtype=torch.int64).view(torch.uint8).to(dec.device))
+    for off in _sync_offsets(dec):
+        dec.arena[off:off + 8].copy_(torch.tensor([value], dtype=torch.int64).view(torch.uint8).to(dec.device))
     torch.cuda.synchronize(dec.device)
 
 
 def _read_sync_counter(dec):
-    off = dec._arena_ptr - dec.arena.data_ptr() + dec.info().ctl_offset
+    """The counter; every copy holds the same count once a launch has ended."""
     torch.cuda.synchronize(dec.device)
-    return int(dec.arena[off:off + 8].cpu().view(torch.int64)[0])
+    vals = [int(dec.arena[off:off + 8].cpu().view(torch.int64)[0]) for off in _sync_offsets(dec)]
+    assert len(set(vals)) == 1, vals
+    return vals[0]
 
 
 @pytest.mark.parametrize("start", [(1 << 32) - 3, (1 << 48) - 5])
@@ -269,6 +277,22 @@ def test_sync_counter_crossing_large_values(kd, start):
     n = compare_gpu_runs(ref, toks.cpu().numpy(), lg[w.prompt_len - 1:], "counter preset",
                          lg2.cpu().numpy()[w.prompt_len - 1:])
     assert n == w.n_gen
+
+
+def test_sync_counter_has_a_copy_on_each_die(kd):
+    """kd_create measures which die owns which counter word and keeps one copy per die
+    (a B200 has two); every CTA adds to both, so both hold the same count after a launch."""
+    w = synth.get("tiny")
+    W = weights_for("tiny")
+    dec = make_decoder(kd, w, W)
+    info = dec.info()
+    assert info.sync_replicas == 2, "one copy only: the probe found a single die"
+    assert info.sync_offset[0] != info.sync_offset[1]
+    assert all((dec._arena_ptr + info.sync_offset[i]) % 2048 == 0 for i in range(2))  # whole die-ownership blocks
+    dec.reset(synth.make_prompt(w).numpy(), 0)
+    dec.decode(8)
+    dec.sync()
+    assert _read_sync_counter(dec) % info.grid == 0
 
 
 def test_argmax_ties_pick_the_lowest_index_across_ctas(kd):
