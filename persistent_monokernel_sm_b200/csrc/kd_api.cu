@@ -75,7 +75,7 @@ Layout make_layout(const Dims& d) {
     y.kcache = take(kv);
     y.vcache = take(kv);
     y.kv_bytes = 2 * kv;
-    y.delta = take((size_t)3 * D * 4);                             // split-K sums, 3 rotating buffers
+    y.delta = take((size_t)3 * kSumCopies * D * 4);                // split-K sums, 3 rotating buffers
     y.qkv = take((size_t)d.qkv_rows * 8);                          // tagged q / k / v of the step
     y.rec = take((size_t)kMaxGrid * d.r * (d.hd + 2) * 8);         // tagged attention records
     y.ctl = take((size_t)kCtlWords * 8);

@@ -493,8 +493,9 @@ __device__ __forceinline__ bool sync_wait(const Smem& sm, const Params& P, const
 __device__ __forceinline__ void zero_previous(const Params& P, long long k) {
     if (k < 1) return;
     const int d = P.dm.d;
-    float* old = reinterpret_cast<float*>(const_cast<uint8_t*>(P.arena) + P.lay.delta) + (size_t)((k - 1) % 3) * d;
-    const int z0 = (int)((long long)d * blockIdx.x / P.nb), z1 = (int)((long long)d * (blockIdx.x + 1) / P.nb);
+    const int n = kSumCopies * d;  // every copy of the buffer
+    float* old = reinterpret_cast<float*>(const_cast<uint8_t*>(P.arena) + P.lay.delta) + (size_t)((k - 1) % 3) * n;
+    const int z0 = (int)((long long)n * blockIdx.x / P.nb), z1 = (int)((long long)n * (blockIdx.x + 1) / P.nb);
     for (int i = z0 + (int)threadIdx.x; i < z1; i += kConsumerThreads) old[i] = 0.f;
 }
 // Start copying the norm gain of the coming row GEMV into shared memory (asynchronously:
@@ -511,13 +512,18 @@ __device__ __forceinline__ void prefetch_gain(const Smem& sm, const __nv_bfloat1
 // order, so all of them get the same scale. Also completes the gain prefetch.
 __device__ __forceinline__ float fold_norm(const Smem& sm, const Params& P, long long k) {
     const int d = P.dm.d;
-    const float* src = reinterpret_cast<const float*>(P.arena + P.lay.delta) + (size_t)(k >= 0 ? k % 3 : 0) * d;
+    const float* src = reinterpret_cast<const float*>(P.arena + P.lay.delta) + (size_t)(k >= 0 ? k % 3 : 0) * kSumCopies * d;
     float ss = 0.f;
     for (int i = threadIdx.x * 4; i < d; i += kConsumerThreads * 4) {
         float4* xp = reinterpret_cast<float4*>(sm.x + i);
         float4 x = *xp;
         if (k >= 0) {
-            const float4 v = ld_relaxed_v4(src + i);
+            float4 v = ld_relaxed_v4(src + i);
+#pragma unroll
+            for (int c = 1; c < kSumCopies; ++c) {  // the copies, added in copy order
+                const float4 u = ld_relaxed_v4(src + (size_t)c * d + i);
+                v.x += u.x, v.y += u.y, v.z += u.z, v.w += u.w;
+            }
             x.x += v.x, x.y += v.y, x.z += v.z, x.w += v.w;
             *xp = x;
         }
@@ -1512,7 +1518,8 @@ __global__ void __launch_bounds__(kThreads, 1) monokernel(const __grid_constant_
                 tr.mark(2);
                 int nrows = g.u1 - g.u0;  // down: this CTA's hidden units (sm.hin, from gate/up)
                 if (ph == kO) nrows = g.grp >= 0 ? oproj_inputs<HD>(P, sm, ctl, t, l, ok, tr) : 0;
-                run_splitk(P, sm, ctl, nrows, sm.hin, delta + (size_t)(k % 3) * dm.d, rg, ok, tr);
+                run_splitk(P, sm, ctl, nrows, sm.hin,
+                           delta + ((size_t)(k % 3) * kSumCopies + blockIdx.x % kSumCopies) * dm.d, rg, ok, tr);
                 tr.mark(3);
                 ok = consumer_sync_and(ok);
                 if (ok) sync_arrive(sm);
@@ -1527,11 +1534,11 @@ __global__ void __launch_bounds__(kThreads, 1) monokernel(const __grid_constant_
         // the last one (read by nobody after the launch) too.
         ok = sync_wait(sm, P, ctl, k - 1, ok);
         if (ok) {
-            const int d = dm.d;
-            const int z0 = (int)((long long)d * blockIdx.x / P.nb), z1 = (int)((long long)d * (blockIdx.x + 1) / P.nb);
+            const int n = kSumCopies * dm.d;  // a buffer with all its copies
+            const int z0 = (int)((long long)n * blockIdx.x / P.nb), z1 = (int)((long long)n * (blockIdx.x + 1) / P.nb);
             for (int i = z0 + tid; i < z1; i += kConsumerThreads) {
-                delta[(size_t)((k - 1) % 3) * d + i] = 0.f;
-                if (k >= 2) delta[(size_t)((k - 2) % 3) * d + i] = 0.f;
+                delta[(size_t)((k - 1) % 3) * n + i] = 0.f;
+                if (k >= 2) delta[(size_t)((k - 2) % 3) * n + i] = 0.f;
             }
         }
     }

@@ -74,7 +74,7 @@ extern "C" int kd_decode_noalloc(kd_ctx* ctx, const int32_t* d_tokens, int32_t n
         off = up256(off + bytes);
         return at;
     };
-    const size_t o_delta = take((size_t)3 * dm.d * 4);
+    const size_t o_delta = take((size_t)3 * kSumCopies * dm.d * 4);
     const size_t o_qkv = take((size_t)dm.qkv_rows * 8);
     const size_t o_rec = take((size_t)v.nb * dm.r * (dm.hd + 2) * 8);
     const size_t o_ctl = take((size_t)kCtlWords * 8);
