@@ -36,8 +36,8 @@ SPEC_HBM_GBS = 8000.0          # B200 HBM3e specification
 # at a 4k context, `--workload 2b-4k --n-gen 8`). It holds for the kernel source it was taken on
 # only: when csrc/kd_kernel.cu + csrc/kd_layout.h no longer hash to this SHA-256, traffic is
 # null.
-TRAFFIC_CAPTURE = {"kernel_sha256": "ec508df3ae4685a0249ddbe2b2292417377b44b78bdaf92c1c8d238a2682996f",
-                   "dram_bytes": 32999400000.0 + 126809856.0, "algorithmic_bytes": 32998424576.0}
+TRAFFIC_CAPTURE = {"kernel_sha256": "9fdd173b82b6baa5bdf22701c760f7d1b1ebfd750fe9d636e3feeec5e24355d2",
+                   "dram_bytes": 33000076000.0 + 115910400.0, "algorithmic_bytes": 32998424576.0}
 FALLBACK_HBM_GBS = 6650.0       # an earlier B200 copy measurement, used without a measured peaks file
 
 
