@@ -317,17 +317,18 @@ struct Smem {
     float2* rope;             // (cos, sin) for hd/2 frequencies at this step's position
     float* red;               // reduction scratch (kConsumerWarps * 8)
     float* stats;             // attention running max and sum per q head (2 * kMaxGroup)
-    unsigned long long* u64;  // [0] sync counter base of the launch, [1] syncs waited, [2] best key
+    unsigned long long* u64;  // [0] sync count at launch, [1] the local counter copy, [2] the other copy
     int* flag;                // broadcast slots
     uint64_t* full;           // mbarriers
     uint64_t* empty;
     Geo* geo;
+    Piece* piece;             // this step's attention piece (written at the step start)
 };
 
 // Byte offsets of the shared-memory regions; the ring starts at 0 (1024-aligned), the others
 // on 128-byte boundaries. Used by the kernel and for the launch size.
 struct SmemLayout {
-    size_t ring, x, gain, hin, work, qs, kvc, rope, red, stats, u64, flag, full, empty, geo, total;
+    size_t ring, x, gain, hin, work, qs, kvc, rope, red, stats, u64, flag, full, empty, geo, piece, total;
 };
 __host__ __device__ inline SmemLayout smem_layout(int ns, int d, int hd, int r, int hin_floats, int work_floats) {
     SmemLayout L{};
@@ -352,6 +353,7 @@ __host__ __device__ inline SmemLayout smem_layout(int ns, int d, int hd, int r, 
     L.full = take((size_t)kMaxStages * 8);
     L.empty = take((size_t)kMaxStages * 8);
     L.geo = take(sizeof(Geo));
+    L.piece = take(sizeof(Piece));
     L.total = off;
     return L;
 }
@@ -374,6 +376,7 @@ __device__ __forceinline__ Smem carve(const Params& P, uint8_t* base) {
     s.full = reinterpret_cast<uint64_t*>(base + L.full);
     s.empty = reinterpret_cast<uint64_t*>(base + L.empty);
     s.geo = reinterpret_cast<Geo*>(base + L.geo);
+    s.piece = reinterpret_cast<Piece*>(base + L.piece);
     return s;
 }
 
@@ -556,9 +559,10 @@ __device__ __forceinline__ void gemv_rows(const Params& P, const Smem& sm, const
     const int d = P.dm.d;
     const int gs = P.sh.gs, gr = P.sh.gr;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int lgs = __ffs(gs) - 1;  // gs is a power of 2
     const int sl = warp & (gs - 1);
-    const int rw = warp / gs, rstep = kConsumerWarps / gs;
-    const int slen = d / gs;
+    const int rw = warp >> lgs, rstep = kConsumerWarps >> lgs;
+    const int slen = d >> lgs;
     const size_t rowbytes = (size_t)d * 2;
     const int nst = (nrows + gr - 1) / gr;
 
@@ -663,7 +667,7 @@ __device__ __forceinline__ void gemv_rows(const Params& P, const Smem& sm, const
 // Dispatch on the chunks per lane and units per warp (fixed per model).
 __device__ __forceinline__ void run_rows(const Params& P, const Smem& sm, const unsigned long long* ctl, int nrows,
                                          float scale, Ring& rg, bool& ok, Tracer& tr) {
-    const int nch = P.dm.d / P.sh.gs / 256;
+    const int nch = (P.dm.d >> (__ffs(P.sh.gs) - 1)) >> 8;
     const int gm = P.sh.gm;
     if (gm == 1) {
         switch (nch) {
@@ -826,7 +830,7 @@ __device__ __forceinline__ void run_attention(const Params& P, const Smem& sm, c
     const int r = dm.r;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int p = P.pos0 + t;
-    const Piece pc = piece_geo(P, g.piece, p);
+    const Piece pc = *sm.piece;
     const uint32_t tag = qkv_tag(P, t, l);
     constexpr int PPS = kStageBytes / (2 * HD);     // positions per stage
     constexpr int NQ = HD / 32;                     // quarters of the head dim (32 dims each)
@@ -1427,6 +1431,7 @@ __global__ void __launch_bounds__(kThreads, 1) monokernel(const __grid_constant_
                 tok = -1;
             }
             sm.flag[2] = tok;
+            if (g.grp >= 0) *sm.piece = piece_geo(P, g.piece, p);  // 64-bit divisions, once per step
         }
         if (tid < dm.hd / 2)  // this position's RoPE row (cos, sin per pair)
             sm.rope[tid] = __ldg(reinterpret_cast<const float2*>(P.arena + P.lay.rope) + (size_t)p * (dm.hd / 2) + tid);
