@@ -290,7 +290,8 @@ def summarize_trace(tr, traced_ms):
         live.append(b)
     span_cyc = [b[:, 4].max() - b[:, 1].min() for b in live if len(b)]
     mhz = float(np.median(span_cyc)) / (traced_ms * 1e3)  # SM cycles per microsecond
-    keys = ("wait", "compute", "tail", "stage_wait", "total", "first_stage", "stage_span", "after_last_stage")
+    keys = ("wait", "compute", "tail", "stage_wait", "total", "first_stage", "stage_span", "after_last_stage",
+            "gap_before")
     per = {n: {k: [] for k in keys} for n in PHASES}
     spans, boundary, other_gaps, sync_wait, xchg_wait, stage_wait, tails = [], [], [], [], [], [], []
     for b in live:
@@ -320,6 +321,10 @@ def summarize_trace(tr, traced_ms):
         after_sync = ((phs == 0) & (lays > 0)) | (phs == 3) | (phs == 5)
         gaps = (bs[1:, 1] - bs[:-1, 4]) / mhz
         new_step = sts[1:] != sts[:-1]
+        for k, n in enumerate(PHASES):  # the gap from the previous phase of the same step
+            m = (phs[1:] == k) & ~new_step
+            if m.any():
+                per[n]["gap_before"].append(gaps[m].mean())
         nsteps = max(1, len(set(sts.tolist())) - 1)
         boundary.append(gaps[new_step].sum() / nsteps)
         other_gaps.append(gaps[~new_step].sum() / nsteps)

@@ -43,6 +43,8 @@ def test_summary_of_a_known_trace():
         assert p["tail"] == pytest.approx(1.0)
         assert p["stage_wait"] == pytest.approx(1.0)
         assert p["total"] == pytest.approx(8.0)
+        if n != "qkv":
+            assert p["gap_before"] == pytest.approx(0.0)
     # steps 1..3: 11 phases each; sync-gated waits: Q/K/V of layer >= 1, gate/up, LM head
     nph = 5 * layers + 1
     span = 3 * nph * 8 + 2 * 3
