@@ -36,8 +36,8 @@ SPEC_HBM_GBS = 8000.0          # B200 HBM3e specification
 # at a 4k context, `--workload 2b-4k --n-gen 8`). It holds for the kernel source it was taken on
 # only: when csrc/kd_kernel.cu + csrc/kd_layout.h no longer hash to this SHA-256, traffic is
 # null.
-TRAFFIC_CAPTURE = {"kernel_sha256": "9fdd173b82b6baa5bdf22701c760f7d1b1ebfd750fe9d636e3feeec5e24355d2",
-                   "dram_bytes": 33000076000.0 + 115910400.0, "algorithmic_bytes": 32998424576.0}
+TRAFFIC_CAPTURE = {"kernel_sha256": "efaf1d0e896a67aa36f43a875fd0f36be8d1676f0e8d5d55460efc867972b010",
+                   "dram_bytes": 32997504000.0 + 169475840.0, "algorithmic_bytes": 32998424576.0}
 FALLBACK_HBM_GBS = 6650.0       # an earlier B200 copy measurement, used without a measured peaks file
 
 
