@@ -25,7 +25,7 @@ def test_one_round_places_the_products_as_defined():
 
 
 def test_key_is_bumped_between_rounds():
-    # zero counter and key: round 1 leaves zeros, round 2 sees the key bumped once
+    # zero counter and key: the first Philox round leaves zeros, the second sees the key bumped once
     assert _one((0, 0, 0, 0), (0, 0), 1) == (0, 0, 0, 0)
     assert _one((0, 0, 0, 0), (0, 0), 2) == (0x9E3779B9, 0, 0xBB67AE85, 0)
 
