@@ -19,9 +19,10 @@
 //  * Two cross-CTA sums per layer. The output projection and the down projection are
 //    split over their reduction dimension (split-K): each CTA multiplies the attention
 //    output dims or the hidden units it produced itself by the matching transposed weight
-//    rows and adds its partial d-vector into a zeroed buffer with vector atomics, then
-//    arrives on one monotonic 64-bit counter. Every CTA keeps the whole residual stream in
-//    shared memory and folds the sum in once the counter reaches its target.
+//    rows and adds its partial d-vector into one of two zeroed copies of the sum with vector
+//    atomics, then arrives on a monotonic 64-bit counter (one copy of it on each of the
+//    B200's two dies). Every CTA keeps the whole residual stream in shared memory and folds
+//    the sum in once the counter reaches its target.
 //  * Group-local exchanges. The CTAs of one kv head compute that head's Q/K/V rows, its
 //    attention pieces and its output-projection columns, so the Q/K/V -> attention and
 //    attention -> output-projection hand-offs only wait for sibling CTAs. They pass 64-bit
@@ -450,10 +451,9 @@ __device__ __forceinline__ bool get_word(const unsigned long long* p, uint32_t t
     return tagged_is(w, tag) || poll_word(p, tag, w, P, ctl, what);
 }
 
-// Arrive at cross-CTA sync k: every consumer thread's atomics of this phase are done (the
-// CTA barrier), then one release add publishes them with the arrival.
-// Arrive at the next cross-CTA sync: after a CTA barrier, thread 0 adds 1 to every replica of
-// the counter with release semantics (one fence, then the adds).
+// Arrive at the next cross-CTA sync: every consumer thread's atomics of this phase are done
+// (the CTA barrier), then thread 0 publishes them with the arrival: one release fence and an
+// add of 1 on every copy of the counter.
 __device__ __forceinline__ void sync_arrive(const Smem& sm) {
     consumer_sync();
     if (threadIdx.x == 0) {
@@ -509,8 +509,9 @@ __device__ __forceinline__ void prefetch_gain(const Smem& sm, const __nv_bfloat1
 }
 
 // The residual stream's update and its RMSNorm scale. With k >= 0 (sync k has completed),
-// delta buffer k % 3 -- the sum of every CTA's split-K partials -- is folded into the
-// residual first, and this CTA's slice of the previous buffer is recycled. Returns
+// delta buffer k % 3 -- the sum of every CTA's split-K partials, its copies added in copy
+// order -- is folded into the residual first, and this CTA's slice of the previous buffer is
+// recycled. Returns
 // 1 / sqrt(mean(x^2) + eps) of the result: every CTA sums the same values in the same
 // order, so all of them get the same scale. Also completes the gain prefetch.
 __device__ __forceinline__ float fold_norm(const Smem& sm, const Params& P, long long k) {
