@@ -348,6 +348,26 @@ def summarize_trace(tr, traced_ms):
     }
 
 
+def read_stream_gbs(device, gib: int = 4, reps: int = 3) -> float:
+    """Read-only HBM bandwidth for context beside the copy-based peak: the best of `reps`
+    timed sums over a `gib` GiB bf16 buffer (a library reduction, outside the timed region of
+    the decode)."""
+    import torch
+    buf = torch.ones(gib << 29, dtype=torch.bfloat16, device=device)  # gib GiB
+    torch.cuda.synchronize(device)
+    best = float("inf")
+    for _ in range(reps + 1):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        s = buf.sum(dtype=torch.float32)
+        e1.record()
+        torch.cuda.synchronize(device)
+        best = min(best, e0.elapsed_time(e1))
+    del buf, s
+    torch.cuda.empty_cache()
+    return (gib << 30) / (best * 1e-3) / 1e9
+
+
 def workload_config(w, n_gen):
     return {"workload": w.name, "n_layers": w.n_layers, "d_model": w.d_model, "n_heads": w.n_heads,
             "n_kv_heads": w.n_kv_heads, "head_dim": w.head_dim, "ffn_dim": w.ffn_dim, "vocab": w.vocab,
@@ -482,12 +502,14 @@ def main():
                     "h2d_bytes_per_step": 4 * w.n_pending, "d2h_bytes_per_step": 4 * w.n_gen},
             "gpu_launches": launches, "launches_per_token": launches / (args.steps * w.n_gen),
             "clocks": clk.summary(),
+            "stream_read_gbs": read_stream_gbs(dev),
         }
     if rank == 0 and not args.no_cpu_baseline:
         n = max(1, args.cpu_sample_tokens)
         tps, dt = run_oracle_sample(w, weights_h, Kh, Vh, start.numpy(), n)
         line["cpu_baseline"] = {
             "value": tps, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "effective_gbs": tps * bytes_launch / w.n_gen / 1e9,
             "sample": "first %d greedy tokens of workload %s, single-threaded oracle, %.1f s; host %s, %d cores"
                       % (n, w.name, dt, lscpu_model(), cpu_cores())}
     if rank == 0:
