@@ -17,8 +17,8 @@
  * pairs (i, i+hd/2), frequency theta^(-2i/hd), absolute positions) -> bf16 KV-cache append
  * -> GQA attention (q head h reads kv head h*Hkv/Hq, scale 1/sqrt(hd)) -> output
  * projection + residual -> RMSNorm -> SwiGLU FFN (silu(gate) * up, then down) + residual;
- * then a final RMSNorm, an untied LM head and a greedy argmax (lowest index wins a tie).
- * No biases. Weights and KV cache are bf16; all activations and accumulations are fp32.
+ * then a final RMSNorm, an untied LM head and a greedy argmax (lowest index wins a tie), or,
+ * after kd_set_sampling, a draw from softmax(logits / T) made inside the kernel. No biases. Weights and KV cache are bf16; all activations and accumulations are fp32.
  *
  * Memory ownership. The caller allocates every byte of device memory: one arena of
  * kd_arena_bytes() bytes (weights in the library's streaming layout, the KV cache,
@@ -27,7 +27,8 @@
  * only the host-side handle, freed by kd_destroy.
  *
  * Streams and threads. Every call that touches the device is asynchronous on the stream
- * given to kd_create, except kd_sync and kd_generate, which wait for it. A handle is not
+ * given to kd_create, except kd_sync and kd_generate, which wait for it, and kd_create
+ * itself, which waits once for a short probe of which B200 die owns which control word. A handle is not
  * thread-safe: use one handle per host thread and stream. kd_decode makes exactly one
  * kernel launch (a cooperative launch of one CTA per SM).
  *
