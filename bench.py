@@ -36,8 +36,8 @@ SPEC_HBM_GBS = 8000.0          # B200 HBM3e specification
 # at a 4k context, `--workload 2b-4k --n-gen 8`). It holds for the kernel source it was taken on
 # only: when csrc/kd_kernel.cu + csrc/kd_layout.h no longer hash to this SHA-256, traffic is
 # null.
-TRAFFIC_CAPTURE = {"kernel_sha256": "521f1e799f3879f9d8a370bec02774762cdd6a7adabb0f7cae9e4bb94099c89b",
-                   "dram_bytes": 32997729000.0 + 162188288.0, "algorithmic_bytes": 32998424576.0}
+TRAFFIC_CAPTURE = {"kernel_sha256": "c23556280ff148b3c55673ca72c3471862dbd97e66f81a4b6d581d338a152f88",
+                   "dram_bytes": 32999673000.0 + 163582976.0, "algorithmic_bytes": 32998424576.0}
 FALLBACK_HBM_GBS = 6650.0       # an earlier B200 copy measurement, used without a measured peaks file
 
 

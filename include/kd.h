@@ -165,7 +165,7 @@ int kd_set_timeout(kd_ctx *ctx, int64_t ns);
  * logit_i * (1/temperature) + g_i, g_i = -log(-log(u_i)) (the Gumbel-max rule, an exact draw),
  * in fp32, lowest index on a tie. u_i comes from the counter-based generator Philox4x32-10
  * (Salmon et al., SC 2011) with key (seed mod 2^32, seed div 2^32) and counter
- * (i div 4, position, 0, 0), output word i mod 4, u = (top 24 bits + 0.5) / 2^24; the position is
+ * (i div 4, position, 0, 0), output word i mod 4, u = (top 23 bits + 0.5) / 2^23; the position is
  * the absolute KV position of the step, so a request draws the same tokens however it is split
  * into calls. Logits written to d_logits_out stay the raw logits. Returns KD_EINVAL for a
  * negative or non-finite temperature. */

@@ -14,7 +14,8 @@ and Shaw ("Parallel random numbers: as easy as 1, 2, 3", SC 2011): a 128-bit cou
 0xD2511F53 and 0xCD9E8D57, the key bumped between rounds by 0x9E3779B9 and 0xBB67AE85.
 Stream layout (the same on both sides): key = (seed mod 2^32, seed div 2^32); vocabulary
 index i at absolute position p uses output word i mod 4 of the counter (i div 4, p, 0, 0);
-u = (top 24 bits + 0.5) / 2^24, exact in fp32. The perturbed values are formed in fp32
+u = (top 23 bits + 0.5) / 2^23, exact in fp32 and never 0 or 1 (with 24 bits, k + 0.5 rounds
+for k >= 2^23 and u can reach 1, where g is infinite). The perturbed values are formed in fp32
 (logit * (1/T) + g, 1/T itself an fp32 division), the precision the kernel decides the argmax
 in.
 
@@ -61,7 +62,7 @@ def uniforms(seed: int, pos: int, n: int) -> np.ndarray:
     out = philox4x32((blk, np.full_like(blk, pos & MASK), z, z), (seed & MASK, (seed >> 32) & MASK))
     words = np.stack(out, axis=1)  # [n][4]
     w = words[np.arange(n), (i & np.uint64(3)).astype(np.int64)]
-    return ((w >> np.uint32(8)).astype(np.float32) + np.float32(0.5)) * np.float32(2.0 ** -24)
+    return ((w >> np.uint32(9)).astype(np.float32) + np.float32(0.5)) * np.float32(2.0 ** -23)
 
 
 def gumbel(seed: int, pos: int, n: int) -> np.ndarray:

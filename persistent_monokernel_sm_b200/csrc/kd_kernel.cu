@@ -1331,12 +1331,13 @@ __device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1
     return c;
 }
 // logit * (1/T) + g for vocabulary index i at absolute position pos, g = -log(-log(u)) with u
-// the (i mod 4)-th word of Philox((i div 4, pos, 0, 0), seed): its top 24 bits + 0.5, / 2^24.
+// the (i mod 4)-th word of Philox((i div 4, pos, 0, 0), seed): its top 23 bits + 0.5, / 2^23
+// (exact in fp32, so u is never 0 or 1).
 __device__ __forceinline__ float gumbel_perturbed(const Params& P, float y, int i, int pos) {
     const uint4 w = philox4x32_10(make_uint4((uint32_t)i >> 2, (uint32_t)pos, 0u, 0u), P.seed_lo, P.seed_hi);
     const int q = i & 3;
     const uint32_t x = q == 0 ? w.x : q == 1 ? w.y : q == 2 ? w.z : w.w;
-    const float u = ((float)(x >> 8) + 0.5f) * 5.9604644775390625e-8f;  // 2^-24
+    const float u = ((float)(x >> 9) + 0.5f) * 1.1920928955078125e-7f;  // 2^-23
     return y * P.inv_temp - logf(-logf(u));
 }
 

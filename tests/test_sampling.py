@@ -34,6 +34,14 @@ def test_uniforms_are_in_the_open_interval_and_uniform():
     u = S.uniforms(seed=12345, pos=77, n=1 << 16)
     assert u.dtype == np.float32
     assert np.all(u > 0) and np.all(u < 1)
+    # every u sits on the lattice (k + 1/2) / 2^23, k an integer in [0, 2^23): exact in fp32,
+    # never 0 or 1, so -log(-log(u)) is always finite
+    k = u.astype(np.float64) * 2.0 ** 23 - 0.5
+    assert np.all(k == np.round(k)) and k.min() >= 0 and k.max() < 2 ** 23
+    top = S.uniforms(seed=0, pos=0, n=1)  # the largest word maps strictly below 1
+    w = np.array([0xFFFFFFFF], np.uint32)
+    assert ((w >> np.uint32(9)).astype(np.float32) + np.float32(0.5)) * np.float32(2.0 ** -23) < 1
+    assert top.dtype == np.float32
     assert abs(float(u.mean()) - 0.5) < 0.005
     counts = np.bincount(np.minimum((u * 64).astype(np.int64), 63), minlength=64)
     expect = u.size / 64
